@@ -1,0 +1,9 @@
+"""thdcp: packed-sequence (THD) causal attention with EOD resets under load-balanced
+KV-all-gather context parallelism, as a C-ABI CUDA library for B200 (sm_100a) with a
+thin Python binding.  All context-parallel ranks are virtual ranks on one GPU.
+
+Method: MindSpeed pull request #3820, "feat: kvallgather cp thd load balance".
+"""
+from .api import (Plan, thd_cp_attn_bwd, thd_cp_attn_bwd_workspace, thd_cp_attn_fwd,  # noqa: F401
+                  thd_cp_plan, thd_kv_gather, thd_rows_to_global)
+from ._lib import ThdError, lib  # noqa: F401

@@ -1,0 +1,334 @@
+// C ABI of libthdcp (declared in include/thdcp.h): argument validation, plan
+// lifecycle with cached device tables, TMA descriptor encoding and kernel launches.
+// No entry point falls back to another implementation: an unsupported shape is an
+// error, and every computation runs in this library's kernels.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "kernels.h"
+#include "plan.h"
+#include "sm100.cuh"
+
+namespace {
+
+using thd_plan = thd_cp_plan_s;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_current() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows, heads, dim] bf16 tensor viewed as a 3-D map with 64-column x 1-head x
+// 128-row boxes, 128-byte swizzle (the layout the tcgen05 descriptors expect).
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)dim * 2, (cuuint64_t)heads * dim * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_heads(int32_t hq, int32_t hkv) {
+    if (hq < 1 || hkv < 1 || hq % hkv != 0) return THD_ERR_INVALID_ARG;
+    return THD_OK;
+}
+
+int ready(thd_plan* p) {
+    if (!p) return THD_ERR_INVALID_ARG;
+    if (!p->uploaded) return THD_ERR_NOT_UPLOADED;
+    return THD_OK;
+}
+
+void free_device(thd_plan* p) {
+    int32_t** ptrs[] = {&p->d_q_idx, &p->d_rm_of_global, &p->d_qtiles, &p->d_entries,
+                        &p->d_lpt,   &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt, &p->d_status};
+    for (auto pp : ptrs) {
+        if (*pp) cudaFree(*pp);
+        *pp = nullptr;
+    }
+    p->uploaded = false;
+}
+
+}  // namespace
+
+extern "C" {
+
+int thd_cp_plan(const int32_t* cu_seqlens, int32_t n_docs, int32_t cp, thd_cp_plan_t* out) {
+    if (!out) return THD_ERR_INVALID_ARG;
+    thd_plan* p = new (std::nothrow) thd_plan();
+    if (!p) return THD_ERR_ALLOC;
+    const int rc = thd_build_plan(cu_seqlens, n_docs, cp, p);
+    if (rc != THD_OK) {
+        delete p;
+        return rc;
+    }
+    *out = p;
+    return THD_OK;
+}
+
+int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out) {
+    if (!plan || !out) return THD_ERR_INVALID_ARG;
+    out->T = plan->T;
+    out->cp = plan->cp;
+    out->n_docs = plan->n_docs;
+    out->Tl = plan->Tl;
+    out->n_qtiles = plan->n_qtiles();
+    out->n_entries = plan->n_entries();
+    out->causal_pairs = plan->causal_pairs;
+    return THD_OK;
+}
+
+int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global, int32_t* qtiles,
+                       int32_t* entries, int32_t* lpt, int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt) {
+    if (!plan) return THD_ERR_INVALID_ARG;
+    auto cp = [](int32_t* dst, const std::vector<int32_t>& v) {
+        if (dst && !v.empty()) std::memcpy(dst, v.data(), v.size() * sizeof(int32_t));
+    };
+    cp(q_idx, plan->q_idx);
+    cp(rm_of_global, plan->rm_of_global);
+    cp(qtiles, plan->qtiles);
+    cp(entries, plan->entries);
+    cp(lpt, plan->lpt);
+    cp(kt_off, plan->kt_off);
+    cp(kt_list, plan->kt_list);
+    cp(kt_lpt, plan->kt_lpt);
+    return THD_OK;
+}
+
+int thd_cp_plan_upload(thd_cp_plan_t plan, void* stream) {
+    if (!plan) return THD_ERR_INVALID_ARG;
+    if (plan->uploaded) return THD_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    struct Item {
+        int32_t** dst;
+        const std::vector<int32_t>* src;
+    } items[] = {{&plan->d_q_idx, &plan->q_idx},     {&plan->d_rm_of_global, &plan->rm_of_global},
+                 {&plan->d_qtiles, &plan->qtiles},   {&plan->d_entries, &plan->entries},
+                 {&plan->d_lpt, &plan->lpt},         {&plan->d_kt_off, &plan->kt_off},
+                 {&plan->d_kt_list, &plan->kt_list}, {&plan->d_kt_lpt, &plan->kt_lpt}};
+    for (auto& it : items) {
+        const size_t bytes = std::max<size_t>(it.src->size(), 4) * sizeof(int32_t);
+        if (cudaMalloc(it.dst, bytes) != cudaSuccess) {
+            free_device(plan);
+            return THD_ERR_ALLOC;
+        }
+        if (!it.src->empty() &&
+            cudaMemcpyAsync(*it.dst, it.src->data(), it.src->size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                            s) != cudaSuccess) {
+            free_device(plan);
+            return THD_ERR_CUDA;
+        }
+    }
+    if (cudaMalloc(&plan->d_status, 16) != cudaSuccess) {
+        free_device(plan);
+        return THD_ERR_ALLOC;
+    }
+    if (cudaMemsetAsync(plan->d_status, 0, 16, s) != cudaSuccess) {
+        free_device(plan);
+        return THD_ERR_CUDA;
+    }
+    cudaGetDevice(&plan->device);
+    plan->uploaded = true;
+    return THD_OK;
+}
+
+void thd_cp_plan_destroy(thd_cp_plan_t plan) {
+    if (!plan) return;
+    if (plan->uploaded) {
+        cudaDeviceSynchronize();
+        free_device(plan);
+    }
+    delete plan;
+}
+
+int thd_kv_gather(thd_cp_plan_t plan, const void* k, const void* v, void* k_rm, void* v_rm, int64_t k_row_bytes,
+                  int64_t v_row_bytes, void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!k || !k_rm || k_row_bytes <= 0 || (!v) != (!v_rm) || (v && v_row_bytes <= 0)) return THD_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(k_rm) || (k_row_bytes & 15) || (v && (!aligned16(v) || !aligned16(v_rm))) ||
+        (v && (v_row_bytes & 15)))
+        return THD_ERR_MISALIGNED;
+    if (k_row_bytes / 16 > INT32_MAX || (v && v_row_bytes / 16 > INT32_MAX)) return THD_ERR_INVALID_ARG;
+    if (thd::launch_row_gather(plan->d_q_idx, plan->T, k, k_rm, k_row_bytes, v, v_rm, v_row_bytes,
+                               num_sms_current(), static_cast<cudaStream_t>(stream)))
+        return THD_ERR_CUDA;
+    return THD_OK;
+}
+
+int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst, int64_t row_bytes, void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!src_rm || !dst || row_bytes <= 0) return THD_ERR_INVALID_ARG;
+    if (!aligned16(src_rm) || !aligned16(dst) || (row_bytes & 15)) return THD_ERR_MISALIGNED;
+    if (thd::launch_row_gather(plan->d_rm_of_global, plan->T, src_rm, dst, row_bytes, nullptr, nullptr, 0,
+                               num_sms_current(), static_cast<cudaStream_t>(stream)))
+        return THD_ERR_CUDA;
+    return THD_OK;
+}
+
+int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm, void* o_rm,
+                    float* lse_rm, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale, int32_t dtype,
+                    void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !std::isfinite(scale)) return THD_ERR_INVALID_ARG;
+    if ((rc = check_heads(hq, hkv))) return rc;
+    if (!aligned16(q_rm) || !aligned16(k_rm) || !aligned16(v_rm) || !aligned16(o_rm) || !aligned16(lse_rm))
+        return THD_ERR_MISALIGNED;
+    const int64_t items = plan->n_qtiles() * (int64_t)hq;
+    if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == THD_DTYPE_BF16) {
+        if (!((dqk == 128 && dv == 128) || (dqk == 192 && dv == 128))) return THD_ERR_UNSUPPORTED;
+        CUtensorMap mq, mk, mv;
+        if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
+            !make_map_bf16(&mv, v_rm, plan->T, hkv, dv))
+            return THD_ERR_CUDA;
+        thd::FwdArgs a;
+        a.qtiles = plan->d_qtiles;
+        a.entries = plan->d_entries;
+        a.lpt = plan->d_lpt;
+        a.o = static_cast<__nv_bfloat16*>(o_rm);
+        a.lse = lse_rm;
+        a.hq = hq;
+        a.hkv = hkv;
+        a.T = plan->T;
+        a.scale_log2 = scale * 1.4426950408889634f;
+        a.status = plan->d_status;
+        if (items == 0) return THD_OK;
+        return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, a, (int)items, s) ? THD_ERR_CUDA : THD_OK;
+    }
+    if (dtype == THD_DTYPE_FP32) {
+        if (!((dqk == 64 && dv == 64) || (dqk == 128 && dv == 128))) return THD_ERR_UNSUPPORTED;
+        thd::FwdF32Args a;
+        a.qtiles = plan->d_qtiles;
+        a.entries = plan->d_entries;
+        a.lpt = plan->d_lpt;
+        a.q = static_cast<const float*>(q_rm);
+        a.k = static_cast<const float*>(k_rm);
+        a.v = static_cast<const float*>(v_rm);
+        a.o = static_cast<float*>(o_rm);
+        a.lse = lse_rm;
+        a.hq = hq;
+        a.hkv = hkv;
+        a.T = plan->T;
+        a.scale = scale;
+        if (items == 0) return THD_OK;
+        return thd::launch_fwd_f32(dqk, dv, a, (int)items, s) ? THD_ERR_CUDA : THD_OK;
+    }
+    return THD_ERR_UNSUPPORTED;
+}
+
+int thd_cp_attn_bwd_workspace(thd_cp_plan_t plan, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, int32_t dtype,
+                              size_t* bytes) {
+    if (!plan || !bytes) return THD_ERR_INVALID_ARG;
+    int rc = check_heads(hq, hkv);
+    if (rc) return rc;
+    if (dtype != THD_DTYPE_BF16 || dqk != 128 || dv != 128) return THD_ERR_UNSUPPORTED;
+    const size_t delta = ((size_t)hq * plan->T * sizeof(float) + 255) & ~(size_t)255;
+    *bytes = delta;
+    return THD_OK;
+}
+
+int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm, const void* o_rm,
+                    const float* lse_rm, const void* do_rm, float* dq_rm, float* dk_rm, float* dv_rm,
+                    void* workspace, size_t workspace_bytes, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv,
+                    float scale, int32_t dtype, void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !do_rm || !dq_rm || !dk_rm || !dv_rm || !workspace ||
+        !std::isfinite(scale))
+        return THD_ERR_INVALID_ARG;
+    if ((rc = check_heads(hq, hkv))) return rc;
+    if (dtype != THD_DTYPE_BF16 || dqk != 128 || dv != 128) return THD_ERR_UNSUPPORTED;
+    size_t need = 0;
+    thd_cp_attn_bwd_workspace(plan, hq, hkv, dqk, dv, dtype, &need);
+    if (workspace_bytes < need) return THD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return THD_ERR_MISALIGNED;
+    const void* ptrs[] = {q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, dq_rm, dk_rm, dv_rm};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return THD_ERR_MISALIGNED;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
+        !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !make_map_bf16(&mdo, do_rm, plan->T, hq, dv))
+        return THD_ERR_CUDA;
+    thd::BwdArgs a;
+    a.qtiles = plan->d_qtiles;
+    a.entries = plan->d_entries;
+    a.kt_off = plan->d_kt_off;
+    a.kt_list = plan->d_kt_list;
+    a.kt_lpt = plan->d_kt_lpt;
+    a.o = static_cast<const __nv_bfloat16*>(o_rm);
+    a.dout = static_cast<const __nv_bfloat16*>(do_rm);
+    a.lse = lse_rm;
+    a.delta = static_cast<float*>(workspace);
+    a.dq_acc = dq_rm;
+    a.dk = dk_rm;
+    a.dv = dv_rm;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.T = plan->T;
+    a.scale = scale;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.status = plan->d_status;
+    const int64_t nkt = plan->n_qtiles();
+    if (nkt == 0) return THD_OK;
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, num_sms_current(),
+                                 static_cast<cudaStream_t>(stream))
+               ? THD_ERR_CUDA
+               : THD_OK;
+}
+
+int thd_cp_device_status(thd_cp_plan_t plan, int32_t reset, int32_t* status) {
+    if (!plan || !status) return THD_ERR_INVALID_ARG;
+    if (!plan->uploaded) return THD_ERR_NOT_UPLOADED;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, plan->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return THD_ERR_CUDA;
+    *status = v;
+    if (reset && cudaMemset(plan->d_status, 0, sizeof(int32_t)) != cudaSuccess) return THD_ERR_CUDA;
+    return THD_OK;
+}
+
+const char* thd_cp_strerror(int code) {
+    switch (code) {
+        case THD_OK: return "ok";
+        case THD_ERR_INVALID_ARG: return "invalid argument";
+        case THD_ERR_BAD_SEQLENS: return "cu_seqlens must start at 0 and every document must be non-empty";
+        case THD_ERR_NOT_DIVISIBLE: return "every document length must be divisible by 2 * cp";
+        case THD_ERR_MISALIGNED: return "pointers and row sizes must be multiples of 16 bytes";
+        case THD_ERR_NOT_UPLOADED: return "plan tables are not on the device: call thd_cp_plan_upload";
+        case THD_ERR_CUDA: return "CUDA runtime or launch error";
+        case THD_ERR_UNSUPPORTED: return "unsupported dtype / head dimension combination";
+        case THD_ERR_ALLOC: return "allocation failed";
+        default: return "unknown error";
+    }
+}
+
+}  // extern "C"

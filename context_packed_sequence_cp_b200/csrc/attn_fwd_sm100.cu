@@ -1,0 +1,300 @@
+// Forward causal attention over the rank-major buffers on sm_100a tensor cores.
+//
+// Method: MindSpeed pull request #3820, "feat: kvallgather cp thd load balance",
+// section "What this PR does / why we need it?": one fused attention call covers
+// every document and every context-parallel rank, reading K/V in place in the
+// rank-major (all-gathered) layout, driven by cached per-tile metadata; MHA, GQA
+// and expanded MLA.  Section "Does this PR introduce any user-facing change?":
+// causal attention with EOD reset.
+//
+// One CTA computes one (query tile, query head) work item, items taken in
+// longest-first order.  Warp roles (192 threads):
+//   warp 0      TMA producer: Q tile once, then K and V of every listed entry
+//               into a two-stage ring (128-byte swizzled boxes of 64 columns).
+//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
+//               score buffers, then O += P_{j-1} V_{j-1} with P read from TMEM.
+//   warps 2-5   softmax warpgroup, one query row per thread: reads S_j from TMEM,
+//               masks PARTIAL entries only, keeps the running max / sum in fp32
+//               (base-2, scale folded in), writes P_j as bf16 over S_j, and
+//               rescales O in TMEM only when the running max grows by more than
+//               2^8 (lazy correction); finally O / l and lse to global memory.
+// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,256+DV) O.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace thd {
+namespace {
+
+constexpr int BM = 128, BN = 128, NST = 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int DQK, int DV>
+struct FwdLayout {
+    static constexpr int kBox = BM * 128;  // one 64-column, 128-row swizzled box: 16 KB
+    static constexpr int kQBytes = BM * DQK * 2;
+    static constexpr int kKBytes = BN * DQK * 2;
+    static constexpr int kVBytes = BN * DV * 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + NST * kKBytes;
+    static constexpr int kOffBar = kOffV + NST * kVBytes;
+    static constexpr int kBytes = kOffBar + 256;
+    static constexpr int kDynSmem = kBytes + 1024;  // slack for 1024-byte alignment
+    static_assert(kDynSmem <= 232448, "shared memory budget");
+};
+
+struct Bars {
+    uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2], o_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Number of leading key columns of an entry visible to a query at global position
+// qpos: key t sits at kpos0 + t + (t >= kbrk ? kjump : 0), positions increase with
+// t, so the visible keys are a prefix of the nvalid listed ones.
+__device__ __forceinline__ int visible_prefix(int qpos, int nvalid, int kpos0, int kbrk, int kjump) {
+    if (qpos < kpos0) return 0;
+    const int a = min(kbrk, qpos - kpos0 + 1);
+    if (a < kbrk || kbrk >= nvalid) return min(a, nvalid);
+    const int b0 = kpos0 + kbrk + kjump;
+    if (qpos < b0) return kbrk;
+    return min(nvalid, kbrk + (qpos - b0 + 1));
+}
+
+template <int DQK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
+    using L = FwdLayout<DQK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    Bars* bars = reinterpret_cast<Bars*>(smem_raw + (base - raw) + L::kOffBar);
+    const uint32_t sQ = base + L::kOffQ, sK = base + L::kOffK, sV = base + L::kOffV;
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x;
+    const int qt = a.lpt[item / a.hq];
+    const int h = item % a.hq;
+    const int g = h / (a.hq / a.hkv);
+    const int* Q = a.qtiles + (size_t)qt * 12;
+    const int row0 = Q[2], m = Q[3], qpos0 = Q[4], qbrk = Q[5], qjump = Q[6];
+    const int nk = Q[8], e0 = Q[9];
+    const int* E = a.entries + (size_t)e0 * 8;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->q_full), 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&bars->k_full[s]), 1);
+            mbar_init(smem_u32(&bars->v_full[s]), 1);
+            mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars->s_full[b]), 1);
+            mbar_init(smem_u32(&bars->p_full[b]), 128);
+        }
+        mbar_init(smem_u32(&bars->o_done), 1);
+        bars->abort = *reinterpret_cast<volatile int*>(a.status);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (bars->abort) return;  // an earlier CTA timed out: do nothing (no TMEM, no copies)
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const uint32_t qf = smem_u32(&bars->q_full);
+            mbar_arrive_expect_tx(qf, L::kQBytes);
+            for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
+            for (int j = 0; j < nk; ++j) {
+                const int st = j % NST;
+                if (j >= NST) mbar_wait(smem_u32(&bars->kv_empty[st]), ((j / NST) - 1) & 1, abort, a.status, 1);
+                const int k0 = E[j * 8 + 0];
+                const uint32_t kf = smem_u32(&bars->k_full[st]), vf = smem_u32(&bars->v_full[st]);
+                mbar_arrive_expect_tx(kf, L::kKBytes);
+                for (int c = 0; c < DQK / 64; ++c)
+                    tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
+                mbar_arrive_expect_tx(vf, L::kVBytes);
+                for (int c = 0; c < DV / 64; ++c)
+                    tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, k0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+            constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
+            mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
+            tc_fence_after();
+            for (int j = 0; j <= nk; ++j) {
+                if (j < nk) {
+                    const int st = j % NST, b = j & 1;
+                    mbar_wait(smem_u32(&bars->k_full[st]), (j / NST) & 1, abort, a.status, 3);
+                    tc_fence_after();
+                    const uint32_t kb = sK + st * L::kKBytes;
+#pragma unroll
+                    for (int kk = 0; kk < DQK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
+                        mma_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
+                               smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
+                    }
+                    mma_commit(smem_u32(&bars->s_full[b]));
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, st = jj % NST, b = jj & 1;
+                    mbar_wait(smem_u32(&bars->p_full[b]), (jj >> 1) & 1, abort, a.status, 4);
+                    mbar_wait(smem_u32(&bars->v_full[st]), (jj / NST) & 1, abort, a.status, 5);
+                    tc_fence_after();
+                    const uint32_t vb = sV + st * L::kVBytes;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_ts(tmem + 256, tmem + b * 128 + kk * 8,
+                               smem_desc_sw128(vb + kk * 2048, L::kBox, 1024), idPV, (jj > 0 || kk > 0));
+                    mma_commit(smem_u32(&bars->o_done));
+                    if (jj + NST < nk) mma_commit(smem_u32(&bars->kv_empty[st]));  // producer reuses stage
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------------- softmax warpgroup
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const int qpos = qpos0 + row + (row >= qbrk ? qjump : 0);
+        const float sl2 = a.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int j = 0; j < nk; ++j) {
+            const int b = j & 1;
+            mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 6);
+            tc_fence_after();
+            const int nvalid = E[j * 8 + 1];
+            const int cls = E[j * 8 + 5];
+            int cnt = nvalid;
+            if (cls != 2) cnt = visible_prefix(qpos, nvalid, E[j * 8 + 2], E[j * 8 + 3], E[j * 8 + 4]);
+
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + b * 128 + c * 32, sr[c]);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    float v = __uint_as_float(sr[c][t]) * sl2;
+                    v = (c * 32 + t < cnt) ? v : -INFINITY;
+                    sr[c][t] = __float_as_uint(v);
+                    mx = fmaxf(mx, v);
+                }
+            const float m_new = fmaxf(m_run, mx);
+            const bool grow = m_new > m_run + kRescaleThreshold;
+            const float m_use = grow ? m_new : m_run;
+            const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
+            const float alpha = grow ? ex2(m_run - m_safe) : 1.f;
+            float sum = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const int c = half * 2 + c2;
+                        const float p0 = ex2(__uint_as_float(sr[c][t]) - m_safe);
+                        const float p1 = ex2(__uint_as_float(sr[c][t + 1]) - m_safe);
+                        sum += p0 + p1;
+                        pk[c2 * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
+                    }
+                tmem_st32(tmem + lane_addr + b * 128 + half * 32, pk);
+            }
+            l_run = l_run * alpha + sum;
+            m_run = m_use;
+            if (j >= 1) {
+                // PV_{j-1} must be complete before O is touched or PV_j is issued.
+                mbar_wait(smem_u32(&bars->o_done), (j - 1) & 1, abort, a.status, 7);
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                    for (int c = 0; c < DV / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                        tmem_st32(tmem + lane_addr + 256 + c * 32, o);
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_full[b]));
+        }
+        // ---------------------------------------------------- epilogue
+        if (nk > 0) mbar_wait(smem_u32(&bars->o_done), (nk - 1) & 1, abort, a.status, 8);
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16* orow = a.o + ((size_t)(row0 + row) * a.hq + h) * DV;
+#pragma unroll
+        for (int c = 0; c < DV / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                pk[t] = pack_bf16x2(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
+            if (row < m) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+        }
+        if (row < m) a.lse[(size_t)h * a.T + row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int DQK, int DV>
+int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const FwdArgs& a, int n_items,
+           cudaStream_t stream) {
+    using L = FwdLayout<DQK, DV>;
+    static bool configured = false;  // attribute is per device function; idempotent
+    if (!configured) {
+        if (cudaFuncSetAttribute(fwd_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::kDynSmem) != cudaSuccess)
+            return -1;
+        configured = true;
+    }
+    fwd_kernel<DQK, DV><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, a);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                     const FwdArgs& a, int n_items, cudaStream_t stream) {
+    if (dqk == 128 && dv == 128) return launch<128, 128>(q, k, v, a, n_items, stream);
+    if (dqk == 192 && dv == 128) return launch<192, 128>(q, k, v, a, n_items, stream);
+    return -2;
+}
+
+}  // namespace thd

@@ -1,0 +1,70 @@
+// Launch interfaces between the C ABI layer (api.cu) and the device kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace thd {
+
+// ---- row gather (all-gather layout, and its inverse) -----------------------
+// dst_t[j] = src_t[idx[j]] for whole rows of row_bytes_t bytes, t = 0, 1 (the second
+// pair may be null).  Rows are copied with 16-byte vectors.
+int launch_row_gather(const int32_t* idx, int64_t rows, const void* src0, void* dst0, int64_t row_bytes0,
+                      const void* src1, void* dst1, int64_t row_bytes1, int num_sms, cudaStream_t stream);
+
+// ---- forward, bf16 on tcgen05 ----------------------------------------------
+struct FwdArgs {
+    const int32_t* qtiles;
+    const int32_t* entries;
+    const int32_t* lpt;
+    __nv_bfloat16* o;
+    float* lse;
+    int32_t hq, hkv;
+    int64_t T;
+    float scale_log2;  // scale * log2(e)
+    int* status;       // device word: nonzero once a bounded wait gave up
+};
+int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                     const FwdArgs& a, int n_items, cudaStream_t stream);
+
+// ---- forward, fp32 SIMT --------------------------------------------------------
+struct FwdF32Args {
+    const int32_t* qtiles;
+    const int32_t* entries;
+    const int32_t* lpt;
+    const float* q;
+    const float* k;
+    const float* v;
+    float* o;
+    float* lse;
+    int32_t hq, hkv;
+    int64_t T;
+    float scale;
+};
+int launch_fwd_f32(int dqk, int dv, const FwdF32Args& a, int n_items, cudaStream_t stream);
+
+// ---- backward, bf16 on tcgen05 ---------------------------------------------------
+struct BwdArgs {
+    const int32_t* qtiles;
+    const int32_t* entries;
+    const int32_t* kt_off;
+    const int32_t* kt_list;
+    const int32_t* kt_lpt;
+    const __nv_bfloat16* o;
+    const __nv_bfloat16* dout;
+    const float* lse;
+    float* delta;   // [hq, T] workspace
+    float* dq_acc;  // [T, hq, dqk] fp32 workspace / output
+    float* dk;      // [T, hkv, dqk]
+    float* dv;      // [T, hkv, dv]
+    int32_t hq, hkv;
+    int64_t T;
+    float scale;
+    float scale_log2;
+    int* status;
+};
+int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                     const CUtensorMap& dout, const BwdArgs& a, int n_ktiles, int num_sms, cudaStream_t stream);
+
+}  // namespace thd

@@ -1,0 +1,195 @@
+// Host planner of libthdcp: validation, the symmetric two-chunk partition and the
+// cached per-tile metadata, built in closed form.
+//
+// Method: MindSpeed pull request #3820, "feat: kvallgather cp thd load balance".
+// Section "Does this PR introduce any user-facing change?" fixes the input
+// contract (THD packed documents, causal attention with EOD reset, every length a
+// multiple of 2 * cp); section "What this PR does / why we need it?" asks for an
+// EOD-aware symmetric partition, direct rank-major K/V indexing and metadata that
+// is computed once and cached.
+//
+// Partition: document d (start s, length L, chunk c = L / 2cp) is cut into 2cp
+// chunks; rank r keeps chunk r then chunk 2cp-1-r.  Rank r's rows of document d
+// form one contiguous "segment" of 2c rank-major rows starting at
+// r*Tl + s/cp (documents before d contribute 2c' = L'/cp rows each).  Row u of
+// that segment holds global position
+//     u <  c:  s + r c + u
+//     u >= c:  s + (2cp-1-r) c + (u - c).
+// Positions grow with u, so the keys of a segment that a query at position P can
+// see are a prefix; its length is the count of chunk-r keys <= P plus the count of
+// mirror-chunk keys <= P.
+#include "plan.h"
+
+#include <algorithm>
+#include <limits>
+
+namespace {
+
+constexpr int BM = THD_BM;
+constexpr int BN = THD_BN;
+
+struct Layout {
+    int32_t cp;
+    int64_t Tl;
+    const std::vector<int64_t>& s;
+    const std::vector<int64_t>& L;
+    int64_t chunk(int d) const { return L[d] / (2 * cp); }
+    int64_t seg_row(int r, int d) const { return (int64_t)r * Tl + s[d] / cp; }
+    int64_t pos(int r, int d, int64_t u) const {
+        const int64_t c = chunk(d);
+        return u < c ? s[d] + (int64_t)r * c + u : s[d] + (int64_t)(2 * cp - 1 - r) * c + (u - c);
+    }
+    // (pos0, brk, jump) of segment rows u0 .. u0+n-1: pos(t) = pos0 + t + (t >= brk ? jump : 0)
+    void encode(int r, int d, int64_t u0, int64_t n, int32_t* out) const {
+        const int64_t c = chunk(d);
+        out[0] = (int32_t)pos(r, d, u0);
+        out[1] = (int32_t)n;
+        out[2] = 0;
+        const int64_t jump = (int64_t)(2 * cp - 2 - 2 * r) * c;  // gap between chunk r and its mirror
+        if (u0 < c && u0 + n > c && jump != 0) {
+            out[1] = (int32_t)(c - u0);
+            out[2] = (int32_t)jump;
+        }
+    }
+    int64_t visible_prefix(int rk, int d, int64_t pmax) const {
+        const int64_t c = chunk(d);
+        const int64_t a0 = s[d] + (int64_t)rk * c;
+        const int64_t b0 = s[d] + (int64_t)(2 * cp - 1 - rk) * c;
+        const int64_t na = std::clamp<int64_t>(pmax - a0 + 1, 0, c);
+        const int64_t nb = std::clamp<int64_t>(pmax - b0 + 1, 0, c);
+        return na + nb;
+    }
+};
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s* p) {
+    if (!cu || !p || n_docs < 1 || cp < 1) return THD_ERR_INVALID_ARG;
+    if (cu[0] != 0) return THD_ERR_BAD_SEQLENS;
+    std::vector<int64_t> s(n_docs), L(n_docs);
+    for (int d = 0; d < n_docs; ++d) {
+        s[d] = cu[d];
+        L[d] = (int64_t)cu[d + 1] - (int64_t)cu[d];
+        if (L[d] <= 0) return THD_ERR_BAD_SEQLENS;
+    }
+    for (int d = 0; d < n_docs; ++d)
+        if (L[d] % (2 * (int64_t)cp) != 0) return THD_ERR_NOT_DIVISIBLE;
+    const int64_t T = cu[n_docs];
+    const int64_t Tl = T / cp;
+    const Layout lay{cp, Tl, s, L};
+
+    try {
+        p->T = T;
+        p->Tl = Tl;
+        p->cp = cp;
+        p->n_docs = n_docs;
+        p->doc_start = s;
+        p->doc_len = L;
+        p->causal_pairs = 0;
+        for (int d = 0; d < n_docs; ++d) p->causal_pairs += L[d] * (L[d] + 1) / 2;
+
+        // ---- partition ------------------------------------------------------
+        p->q_idx.assign(T, 0);
+        p->rm_of_global.assign(T, 0);
+        for (int r = 0; r < cp; ++r)
+            for (int d = 0; d < n_docs; ++d) {
+                const int64_t base = lay.seg_row(r, d), n = 2 * lay.chunk(d);
+                for (int64_t u = 0; u < n; ++u) {
+                    const int64_t g = lay.pos(r, d, u);
+                    p->q_idx[base + u] = (int32_t)g;
+                    p->rm_of_global[g] = (int32_t)(base + u);
+                }
+            }
+
+        // ---- tiles: the 128-row slices of every (rank, document) segment ------
+        std::vector<int64_t> tile_base((size_t)cp * n_docs + 1, 0);
+        for (int r = 0; r < cp; ++r)
+            for (int d = 0; d < n_docs; ++d) {
+                const size_t k = (size_t)r * n_docs + d;
+                tile_base[k + 1] = tile_base[k] + ceil_div(2 * lay.chunk(d), BM);
+            }
+        const int64_t n_tiles = tile_base.back();
+        if (n_tiles > std::numeric_limits<int32_t>::max()) return THD_ERR_INVALID_ARG;
+        p->qtiles.assign((size_t)n_tiles * THD_QTILE_FIELDS, 0);
+        p->entries.clear();
+
+        for (int r = 0; r < cp; ++r)
+            for (int d = 0; d < n_docs; ++d) {
+                const int64_t nseg = 2 * lay.chunk(d);
+                for (int64_t i = 0; i * BM < nseg; ++i) {
+                    const int64_t ti = tile_base[(size_t)r * n_docs + d] + i;
+                    const int64_t u0 = i * BM, m = std::min<int64_t>(BM, nseg - u0);
+                    const int64_t qmin = lay.pos(r, d, u0), qmax = lay.pos(r, d, u0 + m - 1);
+                    int32_t* q = &p->qtiles[(size_t)ti * THD_QTILE_FIELDS];
+                    const int64_t first = p->n_entries();
+                    for (int rk = 0; rk < cp; ++rk) {
+                        const int64_t v = lay.visible_prefix(rk, d, qmax);
+                        for (int64_t j = 0; j * BN < v; ++j) {
+                            const int64_t k0u = j * BN, nv = std::min<int64_t>(BN, v - k0u);
+                            int32_t e[THD_ENTRY_FIELDS];
+                            e[0] = (int32_t)(lay.seg_row(rk, d) + k0u);
+                            e[1] = (int32_t)nv;
+                            int32_t enc[3];
+                            lay.encode(rk, d, k0u, nv, enc);
+                            e[2] = enc[0];
+                            e[3] = enc[1];
+                            e[4] = enc[2];
+                            e[5] = lay.pos(rk, d, k0u + nv - 1) <= qmin ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
+                            e[6] = (int32_t)(tile_base[(size_t)rk * n_docs + d] + j);
+                            e[7] = rk;
+                            p->entries.insert(p->entries.end(), e, e + THD_ENTRY_FIELDS);
+                        }
+                    }
+                    int32_t enc[3];
+                    lay.encode(r, d, u0, m, enc);
+                    q[0] = r;
+                    q[1] = d;
+                    q[2] = (int32_t)(lay.seg_row(r, d) + u0);
+                    q[3] = (int32_t)m;
+                    q[4] = enc[0];
+                    q[5] = enc[1];
+                    q[6] = enc[2];
+                    q[7] = (int32_t)qmax;
+                    q[8] = (int32_t)(p->n_entries() - first);
+                    q[9] = (int32_t)first;
+                    q[10] = (int32_t)s[d];
+                    q[11] = (int32_t)(s[d] + L[d]);
+                }
+            }
+        if (p->n_entries() > std::numeric_limits<int32_t>::max() / 2) return THD_ERR_INVALID_ARG;
+
+        // ---- longest-first order of query tiles ------------------------------
+        p->lpt.resize(n_tiles);
+        for (int64_t t = 0; t < n_tiles; ++t) p->lpt[t] = (int32_t)t;
+        std::stable_sort(p->lpt.begin(), p->lpt.end(), [&](int32_t a, int32_t b) {
+            return p->qtiles[(size_t)a * THD_QTILE_FIELDS + 8] > p->qtiles[(size_t)b * THD_QTILE_FIELDS + 8];
+        });
+
+        // ---- key-tile transpose for the backward (counting sort by key tile) --
+        const int64_t ne = p->n_entries();
+        p->kt_off.assign(n_tiles + 1, 0);
+        for (int64_t e = 0; e < ne; ++e) p->kt_off[p->entries[(size_t)e * THD_ENTRY_FIELDS + 6] + 1]++;
+        for (int64_t t = 0; t < n_tiles; ++t) p->kt_off[t + 1] += p->kt_off[t];
+        std::vector<int32_t> fill(p->kt_off.begin(), p->kt_off.end() - 1);
+        p->kt_list.assign((size_t)ne * 2, 0);
+        for (int64_t qt = 0; qt < n_tiles; ++qt) {  // query tiles ascending -> lists sorted
+            const int32_t* q = &p->qtiles[(size_t)qt * THD_QTILE_FIELDS];
+            for (int64_t e = q[9]; e < (int64_t)q[9] + q[8]; ++e) {
+                const int32_t kt = p->entries[(size_t)e * THD_ENTRY_FIELDS + 6];
+                const int32_t at = fill[kt]++;
+                p->kt_list[(size_t)at * 2] = (int32_t)qt;
+                p->kt_list[(size_t)at * 2 + 1] = (int32_t)e;
+            }
+        }
+        p->kt_lpt.resize(n_tiles);
+        for (int64_t t = 0; t < n_tiles; ++t) p->kt_lpt[t] = (int32_t)t;
+        std::stable_sort(p->kt_lpt.begin(), p->kt_lpt.end(), [&](int32_t a, int32_t b) {
+            return p->kt_off[a + 1] - p->kt_off[a] > p->kt_off[b + 1] - p->kt_off[b];
+        });
+    } catch (const std::bad_alloc&) {
+        return THD_ERR_ALLOC;
+    }
+    return THD_OK;
+}

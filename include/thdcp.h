@@ -1,0 +1,226 @@
+/*
+ * thdcp.h -- C ABI of libthdcp: packed-sequence (THD) causal attention with EOD
+ * document-mask resets under load-balanced KV-all-gather context parallelism,
+ * for NVIDIA B200 (sm_100a).  Every context-parallel rank is a virtual rank on one
+ * GPU.
+ *
+ * Source of the method: MindSpeed pull request #3820, "feat: kvallgather cp thd
+ * load balance".
+ *   [WHAT]  section "What this PR does / why we need it?": load-balanced
+ *           KV-all-gather context parallelism for the THD format, EOD-aware
+ *           symmetric sequence partitioning, a THD attention path with direct
+ *           rank-major K/V indexing and one fused attention call, metadata
+ *           caching, and MHA, GQA and expanded MLA head layouts.
+ *   [USER]  section "Does this PR introduce any user-facing change?": THD packed
+ *           sequences, causal attention, EOD attention-mask reset, and every packed
+ *           subsequence length divisible by 2 * context_parallel_size.
+ *
+ * Conventions shared by every entry point
+ *   - Return value: THD_OK (0) or a negative THD_ERR_* code.  On an argument or
+ *     layout error nothing is launched and no output is touched.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Device entry points only enqueue work: they never synchronise and
+ *     never allocate device memory, except thd_cp_plan_upload (see there).
+ *   - Device buffers are owned by the caller; the library reads and writes them
+ *     only inside the enqueued kernels.  Device pointers must be 16-byte aligned
+ *     (THD_ERR_MISALIGNED otherwise).
+ *   - Tensors are dense row-major.  "Rank-major" row j is local row j % Tl of
+ *     virtual rank j / Tl, Tl = T / cp: the order an all-gather of the rank-local
+ *     shards produces.  Global order is the packed THD token order.
+ *   - Thread safety: a plan may be used from several host threads once uploaded;
+ *     creating, uploading and destroying it must not race with its use.
+ */
+#ifndef THDCP_H
+#define THDCP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ------------------------------------------------------- */
+#define THD_OK                 0
+#define THD_ERR_INVALID_ARG   -1  /* null pointer, cp < 1, bad head/dim counts     */
+#define THD_ERR_BAD_SEQLENS   -2  /* cu_seqlens[0] != 0, or a document of length 0  */
+#define THD_ERR_NOT_DIVISIBLE -3  /* a document length is not a multiple of 2*cp    */
+#define THD_ERR_MISALIGNED    -4  /* pointer or row size not a multiple of 16 bytes */
+#define THD_ERR_NOT_UPLOADED  -5  /* device entry point called before plan_upload   */
+#define THD_ERR_CUDA          -6  /* a CUDA runtime call or a launch failed         */
+#define THD_ERR_UNSUPPORTED   -7  /* dtype / head-dim combination not built         */
+#define THD_ERR_ALLOC         -8  /* host or device allocation failed               */
+
+/* ---- element types ----------------------------------------------------- */
+#define THD_DTYPE_BF16 0   /* bf16 inputs, fp32 accumulation, tcgen05 tensor cores */
+#define THD_DTYPE_FP32 1   /* fp32 inputs and arithmetic (exact-precision path)    */
+
+/* Tile geometry of the cached metadata (fixed; part of the plan's contract). */
+#define THD_BM 128
+#define THD_BN 128
+#define THD_QTILE_FIELDS 12
+#define THD_ENTRY_FIELDS 8
+#define THD_CLS_PARTIAL  1
+#define THD_CLS_UNMASKED 2
+
+typedef struct thd_cp_plan_s* thd_cp_plan_t;   /* opaque, library-owned */
+
+typedef struct thd_cp_plan_info_s {
+    int64_t T;          /* packed tokens                                        */
+    int32_t cp;         /* virtual context-parallel ranks                        */
+    int32_t n_docs;     /* documents                                             */
+    int64_t Tl;         /* tokens per rank, T / cp                               */
+    int64_t n_qtiles;   /* 128-row tiles (query tiles == key tiles)              */
+    int64_t n_entries;  /* listed (query tile, key tile) pairs                   */
+    int64_t causal_pairs; /* sum over documents of L (L + 1) / 2                 */
+} thd_cp_plan_info_t;
+
+/*
+ * thd_cp_plan -- validate a packed layout and build the symmetric partition and
+ * the per-tile metadata ([USER] divisibility rule; [WHAT] EOD-aware symmetric
+ * partitioning and metadata caching).
+ *
+ *   cu_seqlens  host int32[n_docs + 1]: document d spans global tokens
+ *               [cu_seqlens[d], cu_seqlens[d+1]).  Documents are EOD-delimited:
+ *               attention never crosses a boundary.
+ *   n_docs      >= 1.
+ *   cp          virtual ranks, >= 1.  Document d (length L, chunk c = L / (2 cp))
+ *               is cut into 2 cp chunks; rank r owns chunk r and chunk 2 cp-1-r,
+ *               documents ascending, chunk r first.
+ *   out         receives a new plan; *out is left untouched on error.
+ *
+ * Errors: THD_ERR_INVALID_ARG (null, n_docs < 1, cp < 1, T overflow),
+ * THD_ERR_BAD_SEQLENS, THD_ERR_NOT_DIVISIBLE, THD_ERR_ALLOC.  Host only.
+ */
+int thd_cp_plan(const int32_t* cu_seqlens, int32_t n_docs, int32_t cp, thd_cp_plan_t* out);
+
+/* Sizes of the plan's tables.  Host only. */
+int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out);
+
+/*
+ * thd_cp_plan_export -- copy the host tables into caller-allocated host arrays;
+ * any pointer may be NULL to skip that table.
+ *   q_idx        int32[T]      global token at rank-major row j
+ *   rm_of_global int32[T]      rank-major row of global token g (inverse)
+ *   qtiles       int32[n_qtiles * 12]: r, d, row0, m, qpos0, qbrk, qjump,
+ *                qpos_max, nk, entry_off, doc_start, doc_end.  Tile rows are
+ *                rank-major rows row0 .. row0+m-1 of one (rank, document) segment;
+ *                the global position of tile row t is
+ *                qpos0 + t + (t >= qbrk ? qjump : 0).
+ *   entries      int32[n_entries * 8]: k0, nvalid, kpos0, kbrk, kjump, cls,
+ *                ktile, key_rank.  Key rows k0 .. k0+nvalid-1 (rank-major, read in
+ *                place: [WHAT] direct rank-major K/V indexing) are the keys of
+ *                one 128-row slice that some row of the query tile can see;
+ *                cls = THD_CLS_UNMASKED when every row sees every key, else
+ *                THD_CLS_PARTIAL.  Fully masked slices are not listed.
+ *   lpt          int32[n_qtiles]   query tiles by descending nk (ties by index)
+ *   kt_off       int32[n_qtiles+1] CSR offsets of the key-tile transpose
+ *   kt_list      int32[n_entries*2] (qtile, entry) per key tile, qtile ascending
+ *   kt_lpt       int32[n_qtiles]   key tiles by descending list length
+ */
+int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global,
+                       int32_t* qtiles, int32_t* entries, int32_t* lpt,
+                       int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt);
+
+/*
+ * thd_cp_plan_upload -- copy the tables to the current device once and keep them
+ * there ([WHAT] metadata caching).  Allocates device memory owned by the plan
+ * (freed by thd_cp_plan_destroy) and enqueues the copies on `stream`; the host
+ * tables stay valid.  Calling it again is a no-op.  Errors: THD_ERR_CUDA,
+ * THD_ERR_ALLOC.
+ */
+int thd_cp_plan_upload(thd_cp_plan_t plan, void* stream);
+
+/* Release the plan and its device tables (synchronises the device first if
+ * tables were uploaded).  NULL is ignored. */
+void thd_cp_plan_destroy(thd_cp_plan_t plan);
+
+/*
+ * thd_kv_gather -- materialise the rank-major buffer an all-gather of the
+ * rank-local K/V shards produces ([WHAT] KV-all-gather, rank-major indexing):
+ *   k_rm[j] = k[q_idx[j]],  v_rm[j] = v[q_idx[j]]   (whole rows, bit copies).
+ * The same call shards Q or dO (pass v = v_rm = NULL).  One launch.
+ *   k, v         device, [T, row] in global order (row = k_row_bytes bytes)
+ *   k_rm, v_rm   device, [T, row] rank-major; must not overlap the sources
+ *   *_row_bytes  > 0 and multiples of 16
+ * Errors: THD_ERR_INVALID_ARG, THD_ERR_MISALIGNED, THD_ERR_NOT_UPLOADED,
+ * THD_ERR_CUDA.
+ */
+int thd_kv_gather(thd_cp_plan_t plan, const void* k, const void* v, void* k_rm, void* v_rm,
+                  int64_t k_row_bytes, int64_t v_row_bytes, void* stream);
+
+/*
+ * thd_rows_to_global -- the inverse permutation: dst[g] = src_rm[rm_of_global[g]],
+ * whole rows of row_bytes bytes (multiple of 16).  Used to return rank-major
+ * outputs in packed order.  Same errors as thd_kv_gather.
+ */
+int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst,
+                       int64_t row_bytes, void* stream);
+
+/*
+ * thd_cp_attn_fwd -- causal attention with EOD resets over the rank-major buffers,
+ * every virtual rank at once, in one launch ([WHAT] single fused attention call;
+ * [USER] causal + EOD reset).  For each rank-major query row i of document d and
+ * query head h (key/value head g = h / (hq / hkv)):
+ *   S_ij = scale * q_rm[i,h,:] . k_rm[j,g,:] over rank-major key rows j of d with
+ *          position(j) <= position(i);
+ *   o_rm[i,h,:]  = sum_j softmax_j(S_ij) v_rm[j,g,:];
+ *   lse_rm[h*T+i] = log sum_j exp(S_ij)   (natural log, fp32).
+ * Tiles the metadata lists as fully masked are never computed; the mask is
+ * applied only on PARTIAL tiles.
+ *   q_rm  [T, hq, dqk], k_rm [T, hkv, dqk], v_rm [T, hkv, dv], o_rm [T, hq, dv]:
+ *         element type `dtype`; lse_rm fp32 [hq, T].
+ *   hq % hkv == 0.  THD_DTYPE_BF16: (dqk, dv) in {(128,128), (192,128)}.
+ *   THD_DTYPE_FP32: (dqk, dv) in {(64,64), (128,128)}.
+ * Errors: THD_ERR_INVALID_ARG, THD_ERR_UNSUPPORTED, THD_ERR_MISALIGNED,
+ * THD_ERR_NOT_UPLOADED, THD_ERR_CUDA.
+ */
+int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm,
+                    void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, int32_t dqk,
+                    int32_t dv, float scale, int32_t dtype, void* stream);
+
+/*
+ * thd_cp_attn_bwd_workspace -- device workspace bytes thd_cp_attn_bwd needs for
+ * these sizes (fp32 row statistics and the fp32 dQ accumulator).
+ */
+int thd_cp_attn_bwd_workspace(thd_cp_plan_t plan, int32_t hq, int32_t hkv, int32_t dqk,
+                              int32_t dv, int32_t dtype, size_t* bytes);
+
+/*
+ * thd_cp_attn_bwd -- gradients of thd_cp_attn_fwd (the backward pass of the
+ * training path the page's context parallelism serves):
+ *   Delta_i = sum(do_i * o_i);  P_ij = exp(S_ij - lse_i) on visible pairs;
+ *   dV_j = sum_{i,h in group} P_ij do_i;   dP_ij = do_i . v_j;
+ *   dS_ij = P_ij (dP_ij - Delta_i);
+ *   dQ_i = scale * sum_j dS_ij k_j;   dK_j = scale * sum_{i,h in group} dS_ij q_i.
+ * Inputs as in the forward (bf16), lse_rm from the forward, do_rm [T, hq, dv]
+ * rank-major.  Outputs dq_rm [T, hq, dqk], dk_rm [T, hkv, dqk], dv_rm [T, hkv, dv]
+ * are fp32, rank-major; dK/dV already hold the sum over virtual ranks (what a
+ * reduce-scatter would deliver).  `workspace` must hold
+ * thd_cp_attn_bwd_workspace bytes, 256-byte aligned; its contents on entry do not
+ * matter.  THD_DTYPE_BF16 with (dqk, dv) = (128, 128) is built.
+ */
+int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm,
+                    const void* o_rm, const float* lse_rm, const void* do_rm,
+                    float* dq_rm, float* dk_rm, float* dv_rm,
+                    void* workspace, size_t workspace_bytes,
+                    int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale,
+                    int32_t dtype, void* stream);
+
+/*
+ * thd_cp_device_status -- every wait inside this library's kernels is bounded
+ * (1 s per wait); a kernel whose wait gives up drains, records a nonzero code in
+ * a status word owned by the plan (allocated by thd_cp_plan_upload) and returns,
+ * so the context stays usable.  This call copies the word into *status (0 = no
+ * timeout since the last reset) and clears it when reset != 0.  It synchronises
+ * the device.  Errors: THD_ERR_INVALID_ARG, THD_ERR_NOT_UPLOADED, THD_ERR_CUDA.
+ */
+int thd_cp_device_status(thd_cp_plan_t plan, int32_t reset, int32_t* status);
+
+/* Static, human-readable text of an error code. */
+const char* thd_cp_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* THDCP_H */

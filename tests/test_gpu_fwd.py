@@ -1,0 +1,104 @@
+"""thd_cp_attn_fwd on the GPU against the fp64 oracle: full comparison where the
+oracle finishes in seconds, sampled rows at the full workload sizes, the
+cp-independence and per-document invariants, and edge layouts."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from context_packed_sequence_cp_b200 import synthetic as syn
+from oracle import attention as A
+from tests.gpu_util import (FP32_MAX, LSE_MAX, assert_bf16_close, run_forward)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_fwd_fp32_tiny_workload():
+    cu, (q, k, v) = syn.workload_inputs(1, 0)
+    o, lse, _, _ = run_forward(cu, 2, q, k, v, scale=1 / math.sqrt(64))
+    want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(64))
+    assert np.abs(o - want_o).max() <= FP32_MAX
+    assert np.abs(lse - want_l).max() <= FP32_MAX
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_fwd_bf16_mha_workload_full(seed):
+    """T=8192, cp=4, MHA 16 heads, D=128: every output compared."""
+    cu, (q, k, v) = syn.workload_inputs(2, seed)
+    o, lse, _, _ = run_forward(cu, 4, q, k, v)
+    want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
+    assert_bf16_close(o, want_o, "O")
+    assert np.abs(lse - want_l).max() <= LSE_MAX
+
+
+def _sample_rows(cu, rng, n_rand=24):
+    rows = set()
+    for d in range(len(cu) - 1):
+        s, e = int(cu[d]), int(cu[d + 1])
+        rows.update({s, e - 1, min(e - 1, s + 127), min(e - 1, s + 128)})
+    rows.update(int(x) for x in rng.integers(0, int(cu[-1]), n_rand))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("cfg", [3, 4, 5])
+def test_fwd_bf16_workload_sampled(cfg):
+    """Full-size GQA (T=32768), expanded MLA (T=65536) and long-context (T=131072)
+    workloads, checked on sampled rows x heads the oracle computes one by one."""
+    w = syn.WORKLOADS[cfg]
+    cu, tens = syn.workload_inputs(cfg, 0)
+    q, k, v = tens[:3]
+    o, lse, _, _ = run_forward(cu, w.cp, q, k, v)
+    rng = np.random.default_rng(cfg)
+    rows = _sample_rows(cu, rng)
+    if cfg == 5:   # the 65536-token document costs 65536 keys per row: keep a subset
+        rows = [r for r in rows if r >= 65536 or r % 97 == 0 or r < 256][:80]
+    heads = sorted({0, w.hq - 1, int(rng.integers(0, w.hq))})
+    want_o, want_l = A.attention_fwd_rows(q, k, v, cu, 1 / math.sqrt(w.dqk), rows, heads)
+    assert_bf16_close(o[rows][:, heads], want_o, "O")
+    assert np.abs(lse[heads][:, rows].T - want_l).max() <= LSE_MAX
+
+
+@pytest.mark.parametrize("hq,hkv,dqk,dv", [(4, 4, 128, 128), (8, 2, 128, 128), (4, 4, 192, 128), (6, 1, 128, 128)])
+@pytest.mark.parametrize("cp", [1, 2, 4, 8])
+def test_fwd_bf16_small_layouts_full(hq, hkv, dqk, dv, cp):
+    """Random layouts spanning several tiles with ragged tails, every output compared."""
+    rng = np.random.default_rng(cp * 31 + hq + dqk)
+    lens = syn.random_lengths(rng, 3000, 2 * cp, max_docs=6) + [2 * cp]   # plus a minimal document
+    cu = syn.cu_seqlens_of(lens)
+    q, k, v = syn.make_tensors(int(cu[-1]), hq, hkv, dqk, dv, torch.bfloat16, seed=cp + hq)
+    o, lse, _, _ = run_forward(cu, cp, q, k, v)
+    want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(dqk))
+    assert_bf16_close(o, want_o, "O")
+    assert np.abs(lse - want_l).max() <= LSE_MAX
+
+
+def test_fwd_bf16_output_independent_of_cp():
+    lens = [512, 2048, 64, 1536]
+    cu = syn.cu_seqlens_of(lens)
+    q, k, v = syn.make_tensors(int(cu[-1]), 4, 2, 128, 128, torch.bfloat16, seed=5)
+    outs = [run_forward(cu, cp, q, k, v)[:2] for cp in (1, 2, 4, 8, 16)]
+    for o, l in outs[1:]:
+        assert np.abs(o - outs[0][0]).max() <= 2e-2
+        assert np.abs(l - outs[0][1]).max() <= LSE_MAX
+
+
+def test_fwd_bf16_each_document_is_standalone_attention():
+    lens = [256, 1024, 32]
+    cu = syn.cu_seqlens_of(lens)
+    q, k, v = syn.make_tensors(int(cu[-1]), 2, 2, 128, 128, torch.bfloat16, seed=8)
+    o, lse, _, _ = run_forward(cu, 4, q, k, v)
+    for d in range(3):
+        s, e = int(cu[d]), int(cu[d + 1])
+        od, ld, _, _ = run_forward(np.array([0, e - s]), 4, q[s:e], k[s:e], v[s:e])
+        assert np.abs(o[s:e] - od).max() <= 2e-2
+        assert np.abs(lse[:, s:e] - ld).max() <= LSE_MAX
+
+
+def test_fwd_rejects_unsupported_dims():
+    import context_packed_sequence_cp_b200 as thd
+    plan = thd.Plan([0, 16], 2).upload()
+    x = torch.zeros(16, 2, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(thd.ThdError) as e:
+        thd.thd_cp_attn_fwd(plan, x, x, x)
+    assert e.value.kind == "UNSUPPORTED"
