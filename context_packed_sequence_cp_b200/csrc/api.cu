@@ -198,7 +198,8 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
                     void* stream) {
     int rc = ready(plan);
     if (rc) return rc;
-    if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !std::isfinite(scale)) return THD_ERR_INVALID_ARG;
+    if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !std::isfinite(scale) || !(scale > 0.f))
+        return THD_ERR_INVALID_ARG;
     if ((rc = check_heads(hq, hkv))) return rc;
     if (!aligned16(q_rm) || !aligned16(k_rm) || !aligned16(v_rm) || !aligned16(o_rm) || !aligned16(lse_rm))
         return THD_ERR_MISALIGNED;
@@ -264,7 +265,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     int rc = ready(plan);
     if (rc) return rc;
     if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !do_rm || !dq_rm || !dk_rm || !dv_rm || !workspace ||
-        !std::isfinite(scale))
+        !std::isfinite(scale) || !(scale > 0.f))
         return THD_ERR_INVALID_ARG;
     if ((rc = check_heads(hq, hkv))) return rc;
     if (dtype != THD_DTYPE_BF16 || dqk != 128 || dv != 128) return THD_ERR_UNSUPPORTED;

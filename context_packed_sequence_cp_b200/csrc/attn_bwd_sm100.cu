@@ -22,13 +22,20 @@
 //                d  dK  += dS^T Q           (A from TMEM)
 //                e  dQp  = dS K             (smem x smem)            -> TMEM A
 //              and dQp is added to the fp32 dQ in global memory with vector
-//              reductions.  dK, dV stay in TMEM for the whole walk and are written
-//              once.
-// Warp roles (320 threads): warp 0 TMA producer (K, V once; Q, dO per step in a
-// two-stage ring), warp 1 TMEM owner and MMA issuer, warps 2-9 two compute
-// warpgroups, each owning half of the 128 columns of every TMEM row.
-// TMEM columns: A [0,128) S^T then dQp; B [128,256) dP^T then P^T (128..191) and
-// dS^T (192..255) as packed bf16; dK [256,384); dV [384,512).
+//              reductions.  Query tiles are walked outer and the group's heads
+//              inner, so CTAs of one group reach the same dQ tiles close together
+//              in time and their reductions meet in L2.  dK, dV stay in TMEM for
+//              the whole walk and are written once.
+// Warp roles (320 threads): warp 0 producer (TMA of K, V once and of Q, dO per step
+// into a two-stage ring; its lanes also stage the step's lse and Delta in shared
+// memory), warp 1 TMEM owner and MMA issuer, warps 2-9 two compute warpgroups,
+// each owning half of the 128 columns of every TMEM row.
+// TMEM columns: A [0,128) S^T, then P^T (0..63) and dS^T (64..127) as packed bf16;
+// B [128,256) dP^T, then dQp; dK [256,384); dV [384,512).
+// Schedule per step: the compute warpgroups form P^T as soon as S^T is in TMEM
+// (phase 1), and dS^T once dP^T is (phase 2); c, d, e follow; S^T of the next step
+// is issued right behind c and d, dP^T of the next step as soon as dQp has been
+// read out, so the exponentials of a step overlap the tensor work of the last.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -50,10 +57,10 @@ struct BwdLayout {
     static constexpr int kOffQ = kOffV + kTile;       // 2 stages
     static constexpr int kOffDO = kOffQ + 2 * kTile;  // 2 stages
     static constexpr int kOffDS = kOffDO + 2 * kTile;
-    static constexpr int kOffStat = kOffDS + kTile;   // lse2[128], delta[128]
-    static constexpr int kOffBar = kOffStat + 1024;
+    static constexpr int kOffStat = kOffDS + kTile;   // 2 stages x (lse2[128], delta[128])
+    static constexpr int kOffBar = kOffStat + 2 * 256 * 4;
     static constexpr int kBytes = kOffBar + 256;
-    static constexpr int kDynSmem = kBytes + 1024;    // slack for 1024-byte alignment
+    static constexpr int kDynSmem = kBytes;           // base is 1024-aligned by declaration (checked)
     static_assert(kDynSmem <= 232448, "shared memory budget");
 };
 
@@ -62,6 +69,27 @@ struct BwdBars {
     uint32_t tmem_base;
     int abort;
 };
+
+// Per-step metadata: the listed (query tile, entry) pair and the fields the step needs.
+struct StepMeta {
+    int row0, m, qpos0, qbrk, qjump, nvalid, cls;
+};
+__device__ __forceinline__ StepMeta load_meta(const BwdArgs& a, int list_pos) {
+    const int2 pr = __ldg(reinterpret_cast<const int2*>(a.kt_list) + list_pos);
+    const int4 q = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12));      // r, d, row0, m
+    const int4 q2 = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12) + 1); // qpos0, qbrk, qjump, qmax
+    const int4 e0 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8));     // k0, nvalid, ..
+    const int4 e1 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8) + 1); // kjump, cls, ..
+    StepMeta mt;
+    mt.row0 = q.z;
+    mt.m = q.w;
+    mt.qpos0 = q2.x;
+    mt.qbrk = q2.y;
+    mt.qjump = q2.z;
+    mt.nvalid = e0.y;
+    mt.cls = e1.y;
+    return mt;
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -116,12 +144,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
     using L = BwdLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gbase = smem_raw + (base - raw);
-    BwdBars* bars = reinterpret_cast<BwdBars*>(gbase + L::kOffBar);
-    float* s_lse = reinterpret_cast<float*>(gbase + L::kOffStat);
-    float* s_delta = s_lse + 128;
+    const uint32_t base = smem_u32(smem_raw);
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw + L::kOffBar);
+    float* s_stat = reinterpret_cast<float*>(smem_raw + L::kOffStat);  // [stage][lse2 128 | delta 128]
     const uint32_t sK = base + L::kOffK, sV = base + L::kOffV, sQ = base + L::kOffQ, sDO = base + L::kOffDO,
                    sDS = base + L::kOffDS;
     volatile int* abort = &bars->abort;
@@ -138,7 +163,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->kv_full), 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->qdo_full[s]), 1);
+            mbar_init(smem_u32(&bars->qdo_full[s]), 1 + 32);  // expect_tx arrival + the warp's lse/Delta stores
             mbar_init(smem_u32(&bars->qdo_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars->s_full), 1);
@@ -147,11 +172,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         mbar_init(smem_u32(&bars->dq_full), 1);
         mbar_init(smem_u32(&bars->dq_free), kCompute);
         mbar_init(smem_u32(&bars->acc_done), 1);
-        bars->abort = *reinterpret_cast<volatile int*>(a.status);
+        // the layout needs the 1024-byte alignment the declaration asks for (swizzle atoms)
+        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
+        if (base & 1023u) atomicCAS(a.status, 0, 99);
         fence_mbar_init();
     }
     __syncthreads();
-    if (bars->abort) return;  // an earlier CTA timed out: do nothing
+    if (bars->abort) return;  // misaligned, or an earlier CTA timed out: do nothing
     if (warp == 1) {
         tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
         tmem_relinquish();
@@ -163,8 +190,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t tA = tmem, tB = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
 
     if (warp == 0) {
+        // ---------------------------------------------------- producer warp
+        // lane 0 issues the TMA copies; all 32 lanes stage lse (base 2) and Delta of
+        // the step's 128 query rows, so no compute thread waits on global memory.
+        const float log2e = 1.4426950408889634f;
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -175,19 +205,41 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
                 tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
             }
-            for (int it = 0; it < n_it; ++it) {
-                const int st = it & 1;
-                if (it >= 2) mbar_wait(smem_u32(&bars->qdo_empty[st]), ((it >> 1) - 1) & 1, abort, a.status, 11);
-                const int h = g * group + it / llen;
-                const int qt = a.kt_list[2 * (l0 + it % llen)];
-                const int row0 = a.qtiles[(size_t)qt * 12 + 2];
-                const uint32_t f = smem_u32(&bars->qdo_full[st]);
+        }
+        StepMeta cur = load_meta(a, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        for (int it = 0; it < n_it; ++it) {
+            const int st = it & 1;
+            const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
+            if (hh == 0 && it > 0) {
+                cur = nxt;
+                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+            }
+            const int h = g * group + hh;
+            const int row0 = cur.row0;
+            float lv[4], dv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t row = (int64_t)row0 + lane + 32 * u;
+                lv[u] = row < a.T ? __ldg(a.lse + (int64_t)h * a.T + row) * log2e : 0.f;
+                dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
+            }
+            if (it >= 2) mbar_wait(smem_u32(&bars->qdo_empty[st]), ((it >> 1) - 1) & 1, abort, a.status, 11);
+            const uint32_t f = smem_u32(&bars->qdo_full[st]);
+            if (lane == 0) {
                 mbar_arrive_expect_tx(f, 2 * kTile);
                 for (int c = 0; c < 2; ++c) {
                     tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, f, c * 64, h, row0);
                     tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
                 }
             }
+            float* stat = s_stat + st * 256;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                stat[lane + 32 * u] = lv[u];
+                stat[128 + lane + 32 * u] = dv[u];
+            }
+            mbar_arrive(f);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -195,44 +247,57 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
             constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);   // A TMEM, B MN-major
             constexpr uint32_t idMM = idesc_bf16_f32(128, 128, true, true);    // A, B MN-major
-            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 12);
-            tc_fence_after();
-            for (int it = 0; it < n_it; ++it) {
-                const int st = it & 1;
-                const uint32_t q = sQ + st * kTile, d = sDO + st * kTile;
-                mbar_wait(smem_u32(&bars->qdo_full[st]), (it >> 1) & 1, abort, a.status, 13);
-                tc_fence_after();
-                // b: dP^T = V dO^T  (region B held P^T / dS^T of the previous step, consumed in order)
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tB, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(d + off, 16, 1024), idKK, kk > 0);
-                }
-                mma_commit(smem_u32(&bars->dp_full));
-                // a: S^T = K Q^T into region A, once the previous dQp has been read out
-                if (it >= 1) mbar_wait(smem_u32(&bars->dq_free), (it - 1) & 1, abort, a.status, 14);
-                tc_fence_after();
+            auto issue_s = [&](int st) {  // a: S^T = K Q^T -> A
+                const uint32_t q = sQ + st * kTile;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                     mma_ss(tA, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(q + off, 16, 1024), idKK, kk > 0);
                 }
                 mma_commit(smem_u32(&bars->s_full));
+            };
+            auto issue_dp = [&](int st) {  // b: dP^T = V dO^T -> B
+                const uint32_t d = sDO + st * kTile;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                    mma_ss(tB, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(d + off, 16, 1024), idKK, kk > 0);
+                }
+                mma_commit(smem_u32(&bars->dp_full));
+            };
+            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 12);
+            mbar_wait(smem_u32(&bars->qdo_full[0]), 0, abort, a.status, 13);
+            tc_fence_after();
+            issue_s(0);
+            issue_dp(0);
+            for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
+                const uint32_t q = sQ + st * kTile, d = sDO + st * kTile;
                 mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 15);
                 tc_fence_after();
-                // c: dV += P^T dO ; d: dK += dS^T Q ; e: dQp = dS K
+                // c: dV += P^T dO ; d: dK += dS^T Q  (A operands from region A)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDV, tB + kk * 8, smem_desc_sw128(d + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                    mma_ts(tDV, tA + kk * 8, smem_desc_sw128(d + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDK, tB + 64 + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                    mma_ts(tDK, tA + 64 + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                // e: dQp = dS K -> B (dP^T there was consumed before ds_ready)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tA, smem_desc_sw128(sDS + kk * 2048, kBox, 1024), smem_desc_sw128(sK + kk * 2048, kBox, 1024),
+                    mma_ss(tB, smem_desc_sw128(sDS + kk * 2048, kBox, 1024), smem_desc_sw128(sK + kk * 2048, kBox, 1024),
                            idMM, kk > 0);
                 mma_commit(smem_u32(&bars->dq_full));
                 if (it + 2 < n_it) mma_commit(smem_u32(&bars->qdo_empty[st]));
+                if (it + 1 < n_it) {
+                    const int sn = (it + 1) & 1;
+                    mbar_wait(smem_u32(&bars->qdo_full[sn]), ((it + 1) >> 1) & 1, abort, a.status, 13);
+                    tc_fence_after();
+                    issue_s(sn);  // region A is rewritten only after c and d have read it (issue order)
+                    mbar_wait(smem_u32(&bars->dq_free), it & 1, abort, a.status, 14);
+                    tc_fence_after();
+                    issue_dp(sn);
+                }
             }
             mma_commit(smem_u32(&bars->acc_done));
         }
@@ -241,37 +306,27 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int ct = threadIdx.x - 64;         // 0..255
         const int hf = ct >> 7;                  // column half
         const int wq = warp & 3;
-        const int r = wq * 32 + lane;            // TMEM lane: key row (softmax), query row (dQ)
+        const int r = wq * 32 + lane;            // TMEM lane: key row (phases 1-2), query row (dQ)
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale_log2;
-        const float log2e = 1.4426950408889634f;
         const int kbrk_t = KT[5], kjump_t = KT[6];
         const int kpos_r = KT[4] + r + (r >= kbrk_t ? kjump_t : 0);
+        StepMeta cur = load_meta(a, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a, l0 + 1);
         for (int it = 0; it < n_it; ++it) {
-            const int h = g * group + it / llen;
-            const int qt = a.kt_list[2 * (l0 + it % llen)];
-            const int e = a.kt_list[2 * (l0 + it % llen) + 1];
-            const int* QT = a.qtiles + (size_t)qt * 12;
-            const int row0 = QT[2], m = QT[3], qpos0 = QT[4], qbrk = QT[5], qjump = QT[6];
-            const int* E = a.entries + (size_t)e * 8;
-            const int nvalid = E[1], cls = E[5];
-
-            // stage lse (base 2) and Delta of the step's 128 query rows
-            named_bar_sync(1, kCompute);
-            {
-                const int i = ct & 127;
-                const int64_t row = row0 + i;
-                float v = 0.f;
-                if (row < a.T) v = (ct < 128) ? a.lse[(int64_t)h * a.T + row] * log2e : a.delta[(int64_t)h * a.T + row];
-                if (ct < 128) s_lse[i] = v; else s_delta[i] = v;
+            const int st = it & 1;
+            const int pos = it / group, hh = it - pos * group;       // query tiles outer, heads inner
+            if (hh == 0 && it > 0) {
+                cur = nxt;
+                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
             }
-            named_bar_sync(1, kCompute);
+            const int h = g * group + hh;
+            const int row0 = cur.row0, m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
 
             // visible query columns of this key row: a suffix [lo, m) of the tile
             int lo = 0, hi = m;
-            if (r >= nvalid) hi = 0;
-            else if (cls != 2) {
-                // first query row whose position reaches kpos_r
+            if (r >= cur.nvalid) hi = 0;
+            else if (cur.cls != 2) {
                 const int n1 = min(qbrk, m);
                 if (kpos_r <= qpos0) lo = 0;
                 else if (kpos_r - qpos0 < n1) lo = kpos_r - qpos0;
@@ -280,35 +335,61 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     lo = (kpos_r <= p1) ? n1 : min(m, n1 + (kpos_r - p1));
                 }
             }
+            const float* stat = s_stat + st * 256;
 
+            // ---- phase 1: P^T = exp(S^T - lse) on this thread's 64 query columns
+            mbar_wait(smem_u32(&bars->qdo_full[st]), (it >> 1) & 1, abort, a.status, 16);  // lse/Delta staged
             mbar_wait(smem_u32(&bars->s_full), it & 1, abort, a.status, 16);
-            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 17);
             tc_fence_after();
-            uint32_t pk[32], dk[32];
+            float p[64];
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
-                uint32_t s[32], dp[32];
+                uint32_t sv[32];
                 const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(tA + lane_addr + c0, s);
-                tmem_ld32(tB + lane_addr + c0, dp);
+                tmem_ld32(tA + lane_addr + c0, sv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < 32; t += 2) {
-                    const int i0 = c0 + t, i1 = c0 + t + 1;
-                    float p0 = ex2(fmaf(__uint_as_float(s[t]), sl2, -s_lse[i0]));
-                    float p1 = ex2(fmaf(__uint_as_float(s[t + 1]), sl2, -s_lse[i1]));
-                    p0 = (i0 >= lo && i0 < hi) ? p0 : 0.f;
-                    p1 = (i1 >= lo && i1 < hi) ? p1 : 0.f;
-                    const float d0 = p0 * (__uint_as_float(dp[t]) - s_delta[i0]);
-                    const float d1 = p1 * (__uint_as_float(dp[t + 1]) - s_delta[i1]);
-                    pk[ch * 16 + t / 2] = pack_bf16x2(p0, p1);
-                    dk[ch * 16 + t / 2] = pack_bf16x2(d0, d1);
+                for (int t = 0; t < 32; t += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(stat + c0 + t);
+                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = c0 + t + u;
+                        const float e = ex2(fmaf(__uint_as_float(sv[t + u]), sl2, -lq[u]));
+                        p[ch * 32 + t + u] = (i >= lo && i < hi) ? e : 0.f;
+                    }
                 }
             }
-            // both warpgroups have read dP^T before either overwrites region B
-            named_bar_sync(1, kCompute);
-            tmem_st32(tB + lane_addr + hf * 32, pk);
-            tmem_st32(tB + lane_addr + 64 + hf * 32, dk);
+            named_bar_sync(1, kCompute);  // every S^T read of region A is done before P^T overwrites it
+            {
+                uint32_t pk[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(p[2 * t], p[2 * t + 1]);
+                tmem_st32(tA + lane_addr + hf * 32, pk);
+            }
+
+            // ---- phase 2: dS^T = P^T (dP^T - Delta)
+            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 17);
+            tc_fence_after();
+            uint32_t dk[32];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t dpv[32];
+                const int c0 = hf * 64 + ch * 32;
+                tmem_ld32(tB + lane_addr + c0, dpv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int t = 0; t < 32; t += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(stat + 128 + c0 + t);
+                    const float dq4[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float ds[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) ds[u] = p[ch * 32 + t + u] * (__uint_as_float(dpv[t + u]) - dq4[u]);
+                    dk[ch * 16 + t / 2] = pack_bf16x2(ds[0], ds[1]);
+                    dk[ch * 16 + t / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                }
+            }
+            tmem_st32(tA + lane_addr + 64 + hf * 32, dk);
             // dS (query-major for the dQ product): rows = key r, 128-byte swizzled
             {
                 const uint32_t rowb = sDS + hf * kBox + r * 128;
@@ -321,14 +402,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->ds_ready));
 
-            // dQp rows (TMEM lane = query row r) into the fp32 dQ
+            // ---- dQp rows (TMEM lane = query row r) into the fp32 dQ
             mbar_wait(smem_u32(&bars->dq_full), it & 1, abort, a.status, 18);
             tc_fence_after();
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t q[32];
                 const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(tA + lane_addr + c0, q);
+                tmem_ld32(tB + lane_addr + c0, q);
                 tmem_wait_ld();
                 if (r < m) {
                     float* dst = a.dq_acc + ((int64_t)(row0 + r) * a.hq + h) * kD + c0;

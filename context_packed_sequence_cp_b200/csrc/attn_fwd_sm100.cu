@@ -27,13 +27,17 @@
 namespace thd {
 namespace {
 
-constexpr int BM = 128, BN = 128, NST = 2;
+constexpr int BM = 128, BN = 128, kMaxStages = 3;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int DQK, int DV>
 struct FwdLayout {
+    // K/V ring depth: a stage is held from its load until its PV product retires, so
+    // three stages keep one load in flight ahead of the two tiles in use (D=128);
+    // the 192-wide keys of expanded MLA leave room for two.
+    static constexpr int NST = (DQK + DV <= 256) ? 3 : 2;
     static constexpr int kBox = BM * 128;  // one 64-column, 128-row swizzled box: 16 KB
     static constexpr int kQBytes = BM * DQK * 2;
     static constexpr int kKBytes = BN * DQK * 2;
@@ -48,7 +52,7 @@ struct FwdLayout {
 };
 
 struct Bars {
-    uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[2], p_full[2], o_done;
+    uint64_t q_full, k_full[kMaxStages], v_full[kMaxStages], kv_empty[kMaxStages], s_full[2], p_full[2], o_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -70,6 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
     using L = FwdLayout<DQK, DV>;
+    constexpr int NST = L::NST;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -122,10 +127,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const uint32_t qf = smem_u32(&bars->q_full);
             mbar_arrive_expect_tx(qf, L::kQBytes);
             for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
+            int k0_next = nk > 0 ? __ldg(E) : 0;
             for (int j = 0; j < nk; ++j) {
                 const int st = j % NST;
+                const int k0 = k0_next;
+                if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
                 if (j >= NST) mbar_wait(smem_u32(&bars->kv_empty[st]), ((j / NST) - 1) & 1, abort, a.status, 1);
-                const int k0 = E[j * 8 + 0];
                 const uint32_t kf = smem_u32(&bars->k_full[st]), vf = smem_u32(&bars->v_full[st]);
                 mbar_arrive_expect_tx(kf, L::kKBytes);
                 for (int c = 0; c < DQK / 64; ++c)
@@ -179,35 +186,53 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int qpos = qpos0 + row + (row >= qbrk ? qjump : 0);
         const float sl2 = a.scale_log2;
         float m_run = -INFINITY, l_run = 0.f;
+        // entry record j+1 is fetched while entry j is processed
+        int4 e_lo = make_int4(0, 0, 0, 0), e_hi = make_int4(0, 0, 0, 0);
+        if (nk > 0) {
+            e_lo = __ldg(reinterpret_cast<const int4*>(E));
+            e_hi = __ldg(reinterpret_cast<const int4*>(E) + 1);
+        }
         for (int j = 0; j < nk; ++j) {
             const int b = j & 1;
+            const int4 c_lo = e_lo, c_hi = e_hi;
+            if (j + 1 < nk) {
+                e_lo = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
+                e_hi = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8) + 1);
+            }
+            // record: k0, nvalid, kpos0, kbrk | kjump, cls, ktile, key_rank
+            const int nvalid = c_lo.y;
+            int cnt = nvalid;
+            if (c_hi.y != 2) cnt = visible_prefix(qpos, nvalid, c_lo.z, c_lo.w, c_hi.x);
             mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 6);
             tc_fence_after();
-            const int nvalid = E[j * 8 + 1];
-            const int cls = E[j * 8 + 5];
-            int cnt = nvalid;
-            if (cls != 2) cnt = visible_prefix(qpos, nvalid, E[j * 8 + 2], E[j * 8 + 3], E[j * 8 + 4]);
 
             uint32_t sr[4][32];
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + b * 128 + c * 32, sr[c]);
             tmem_wait_ld();
-            float mx = -INFINITY;
+            // masked scores -> -inf; row max with 8 independent partial maxima (raw units)
+            float pm[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
-                    float v = __uint_as_float(sr[c][t]) * sl2;
-                    v = (c * 32 + t < cnt) ? v : -INFINITY;
+                    float v = __uint_as_float(sr[c][t]);
+                    if (cnt < 128) v = (c * 32 + t < cnt) ? v : -INFINITY;
                     sr[c][t] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
+                    pm[t & 7] = fmaxf(pm[t & 7], v);
                 }
+            const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + kRescaleThreshold;
             const float m_use = grow ? m_new : m_run;
             const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
             const float alpha = grow ? ex2(m_run - m_safe) : 1.f;
-            float sum = 0.f;
+            float ps[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
@@ -216,13 +241,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
                         const int c = half * 2 + c2;
-                        const float p0 = ex2(__uint_as_float(sr[c][t]) - m_safe);
-                        const float p1 = ex2(__uint_as_float(sr[c][t + 1]) - m_safe);
-                        sum += p0 + p1;
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[c][t]), sl2, -m_safe));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[c][t + 1]), sl2, -m_safe));
+                        ps[(t >> 1) & 7] += p0 + p1;
                         pk[c2 * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
                     }
                 tmem_st32(tmem + lane_addr + b * 128 + half * 32, pk);
             }
+            const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
             if (j >= 1) {

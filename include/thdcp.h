@@ -170,7 +170,8 @@ int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst,
  * applied only on PARTIAL tiles.
  *   q_rm  [T, hq, dqk], k_rm [T, hkv, dqk], v_rm [T, hkv, dv], o_rm [T, hq, dv]:
  *         element type `dtype`; lse_rm fp32 [hq, T].
- *   hq % hkv == 0.  THD_DTYPE_BF16: (dqk, dv) in {(128,128), (192,128)}.
+ *   scale > 0 and finite.  hq % hkv == 0.
+ *   THD_DTYPE_BF16: (dqk, dv) in {(128,128), (192,128)}.
  *   THD_DTYPE_FP32: (dqk, dv) in {(64,64), (128,128)}.
  * Errors: THD_ERR_INVALID_ARG, THD_ERR_UNSUPPORTED, THD_ERR_MISALIGNED,
  * THD_ERR_NOT_UPLOADED, THD_ERR_CUDA.
