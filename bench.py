@@ -247,7 +247,7 @@ def run_native(args):
     ws = torch.empty(thd.thd_cp_attn_bwd_workspace(plan, hq=w.hq, hkv=w.hkv, dqk=w.dqk, dv=w.dv),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 6   # gather Q, gather K/V, gather dO, fwd, bwd prep, bwd
+    launches_per_step = 7   # gather Q, gather K/V, gather dO, fwd, bwd prep, dK/dV, dQ
 
     def step(ev=None):
         if ev:
@@ -362,7 +362,7 @@ def run_native(args):
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, cu, args.seed),
-        "roofline": {"kernel": "bwd (thd_cp_attn_bwd: prep + key-major tcgen05 kernel)", "bound": "tensor",
+        "roofline": {"kernel": "bwd (thd_cp_attn_bwd: prep + key-major dK/dV + query-major dQ tcgen05 kernels)", "bound": "tensor",
                      "achieved": bwd_tf, "peak": sustained, "unit": "TFLOP/s", "frac": bwd_tf / sustained,
                      "traffic": traffic, "peak_source": f"bf16_tflops_sustained ({peak_src})",
                      "flops_per_launch": bwd_fl},

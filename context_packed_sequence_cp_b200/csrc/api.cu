@@ -283,6 +283,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     thd::BwdArgs a;
     a.qtiles = plan->d_qtiles;
     a.entries = plan->d_entries;
+    a.lpt = plan->d_lpt;
     a.kt_off = plan->d_kt_off;
     a.kt_list = plan->d_kt_list;
     a.kt_lpt = plan->d_kt_lpt;

@@ -7,35 +7,26 @@
 // dV summed over every rank that read a key (what a reduce-scatter of the gathered
 // gradients delivers; on one GPU the shared buffer already holds the sum).
 //
-// Two kernels:
-//   bwd_prep   Delta_i = sum_d dO_id O_id per (row, head), and dQ := 0.
-//   bwd_kernel one CTA per (key tile, key/value head g), key tiles in longest-first
-//              order; it walks every query head of g's group and every query tile
-//              that lists the key tile (the plan's key-tile transpose).  Per step,
-//              with key rows on TMEM lanes:
-//                a  S^T  = K Q^T            (tcgen05, smem x smem)  -> TMEM A
-//                b  dP^T = V dO^T           (tcgen05, smem x smem)  -> TMEM B
-//                   P^T = exp(S^T - lse), dS^T = P^T (dP^T - Delta), masked on
-//                   PARTIAL entries and ragged tiles; P^T, dS^T as bf16 over dP^T
-//                   in TMEM, dS (bf16) into shared memory
-//                c  dV  += P^T dO           (A from TMEM)
-//                d  dK  += dS^T Q           (A from TMEM)
-//                e  dQp  = dS K             (smem x smem)            -> TMEM A
-//              and dQp is added to the fp32 dQ in global memory with vector
-//              reductions.  Query tiles are walked outer and the group's heads
-//              inner, so CTAs of one group reach the same dQ tiles close together
-//              in time and their reductions meet in L2.  dK, dV stay in TMEM for
-//              the whole walk and are written once.
-// Warp roles (320 threads): warp 0 producer (TMA of K, V once and of Q, dO per step
-// into a two-stage ring; its lanes also stage the step's lse and Delta in shared
-// memory), warp 1 TMEM owner and MMA issuer, warps 2-9 two compute warpgroups,
-// each owning half of the 128 columns of every TMEM row.
-// TMEM columns: A [0,128) S^T, then P^T (0..63) and dS^T (64..127) as packed bf16;
-// B [128,256) dP^T, then dQp; dK [256,384); dV [384,512).
-// Schedule per step: the compute warpgroups form P^T as soon as S^T is in TMEM
-// (phase 1), and dS^T once dP^T is (phase 2); c, d, e follow; S^T of the next step
-// is issued right behind c and d, dP^T of the next step as soon as dQp has been
-// read out, so the exponentials of a step overlap the tensor work of the last.
+// Three kernels, none with atomics:
+//   bwd_prep   Delta_i = sum_d dO_id O_id per (row, head).
+//   dkdv       one CTA per (key tile, key/value head g), key tiles longest-first; it
+//              walks every query tile the plan's key-tile transpose lists (outer) and
+//              every query head of g's group (inner).  Key rows on TMEM lanes:
+//                a  S^T  = K Q^T   -> TMEM A       b  dP^T = V dO^T -> TMEM B
+//                phase 1: P^T = exp(S^T - lse) -> bf16 over S^T (A)
+//                phase 2: dS^T = P^T (dP^T - Delta) -> bf16 over dP^T (B)
+//                c  dV += P^T dO   (A operand from TMEM A)
+//                d  dK += dS^T Q   (A operand from TMEM B)
+//              issued as c(i), a(i+1), d(i), b(i+1): the exponentials of step i+1
+//              run while d(i) and b(i+1) are on the tensor pipe.  dK, dV stay in
+//              TMEM for the whole walk and are written once.
+//   dq         one CTA per (query tile, query head), like the forward: per listed
+//              entry S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - Delta) as bf16
+//              over S, dQ += dS K with the A operand from TMEM; written once.
+// Recomputing S and dP in the dq kernel costs 3/5 more tensor work than a single
+// kernel that reduces partial dQ tiles into global memory, but the reductions of
+// the single kernel move 64 KB per (query tile, key tile, head) through L2 and cap
+// at the L2's reduction bandwidth once dQ outgrows L2.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -45,41 +36,26 @@ namespace thd {
 namespace {
 
 constexpr int kD = 128;                 // head dim built (Dqk = Dv = 128)
-constexpr int kThreads = 320;
-constexpr int kCompute = 256;           // threads of the two compute warpgroups
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBox = 128 * 128;         // one 64-column x 128-row bf16 box, 16 KB
 constexpr int kTile = 2 * kBox;         // 128 x 128 bf16 tile, 32 KB
+constexpr int kCompute = 256;           // two compute warpgroups
+constexpr int kThreads = 64 + kCompute; // producer warp, MMA warp, compute
 
-struct BwdLayout {
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = kOffK + kTile;
-    static constexpr int kOffQ = kOffV + kTile;       // 2 stages
-    static constexpr int kOffDO = kOffQ + 2 * kTile;  // 2 stages
-    static constexpr int kOffDS = kOffDO + 2 * kTile;
-    static constexpr int kOffStat = kOffDS + kTile;   // 2 stages x (lse2[128], delta[128])
-    static constexpr int kOffBar = kOffStat + 2 * 256 * 4;
-    static constexpr int kBytes = kOffBar + 256;
-    static constexpr int kDynSmem = kBytes;           // base is 1024-aligned by declaration (checked)
-    static_assert(kDynSmem <= 232448, "shared memory budget");
-};
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
-struct BwdBars {
-    uint64_t kv_full, qdo_full[2], qdo_empty[2], s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
-    uint32_t tmem_base;
-    int abort;
-};
-
-// Per-step metadata: the listed (query tile, entry) pair and the fields the step needs.
+// Per-step metadata of the key-major walk: the listed (query tile, entry) pair.
 struct StepMeta {
     int row0, m, qpos0, qbrk, qjump, nvalid, cls;
 };
 __device__ __forceinline__ StepMeta load_meta(const BwdArgs& a, int list_pos) {
     const int2 pr = __ldg(reinterpret_cast<const int2*>(a.kt_list) + list_pos);
     const int4 q = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12));      // r, d, row0, m
-    const int4 q2 = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12) + 1); // qpos0, qbrk, qjump, qmax
-    const int4 e0 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8));     // k0, nvalid, ..
-    const int4 e1 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8) + 1); // kjump, cls, ..
+    const int4 q2 = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12) + 1); // qpos0, qbrk, qjump, -
+    const int4 e0 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8));     // k0, nvalid, -, -
+    const int4 e1 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8) + 1); // kjump, cls, -, -
     StepMeta mt;
     mt.row0 = q.z;
     mt.m = q.w;
@@ -91,29 +67,25 @@ __device__ __forceinline__ StepMeta load_meta(const BwdArgs& a, int list_pos) {
     return mt;
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+// Number of leading key columns of an entry a query at position qpos can see
+// (key t sits at kpos0 + t + (t >= kbrk ? kjump : 0); positions grow with t).
+__device__ __forceinline__ int visible_keys(int qpos, int nvalid, int kpos0, int kbrk, int kjump) {
+    if (qpos < kpos0) return 0;
+    const int a = min(kbrk, qpos - kpos0 + 1);
+    if (a < kbrk || kbrk >= nvalid) return min(a, nvalid);
+    const int b0 = kpos0 + kbrk + kjump;
+    if (qpos < b0) return kbrk;
+    return min(nvalid, kbrk + (qpos - b0 + 1));
 }
 
 // ---------------------------------------------------------------- prep
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
-                                                       float* __restrict__ delta, float4* __restrict__ dq,
-                                                       int64_t rows, int hq, int64_t T, int64_t dq_vec4) {
+                                                       float* __restrict__ delta, int64_t rows, int hq, int64_t T) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * 8;
     for (int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); w < rows; w += nwarps) {
-        // w = row * hq + h, rows of kD bf16 values: 4 per lane
+        // w = row * hq + h; a row holds kD bf16 values, 4 per lane
         const uint2 a = *reinterpret_cast<const uint2*>(o + w * kD + lane * 4);
         const uint2 b = *reinterpret_cast<const uint2*>(dout + w * kD + lane * 4);
         const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
@@ -127,28 +99,38 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) {
-            const int64_t row = w / hq;
-            const int h = (int)(w % hq);
-            delta[(int64_t)h * T + row] = s;
-        }
+        if (lane == 0) delta[(int64_t)(w % hq) * T + w / hq] = s;
     }
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < dq_vec4; i += (int64_t)gridDim.x * blockDim.x)
-        dq[i] = z;
 }
 
-// ---------------------------------------------------------------- main kernel
+// ================================================================ dK / dV
+struct DkdvLayout {
+    static constexpr int kQStages = 3, kDOStages = 2;
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kTile;
+    static constexpr int kOffQ = kOffV + kTile;
+    static constexpr int kOffDO = kOffQ + kQStages * kTile;
+    static constexpr int kOffStat = kOffDO + kDOStages * kTile;  // per dO stage: lse2[128], delta[128]
+    static constexpr int kOffBar = kOffStat + kDOStages * 256 * 4;
+    static constexpr int kBytes = kOffBar + 256;
+    static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+struct DkdvBars {
+    uint64_t kv_full, q_full[3], q_empty[3], do_full[2], do_empty[2], s_full, dp_full, p_ready, ds_ready, acc_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
-    using L = BwdLayout;
+dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
+    using L = DkdvLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
-    BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw + L::kOffBar);
-    float* s_stat = reinterpret_cast<float*>(smem_raw + L::kOffStat);  // [stage][lse2 128 | delta 128]
-    const uint32_t sK = base + L::kOffK, sV = base + L::kOffV, sQ = base + L::kOffQ, sDO = base + L::kOffDO,
-                   sDS = base + L::kOffDS;
+    DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem_raw + L::kOffBar);
+    float* s_stat = reinterpret_cast<float*>(smem_raw + L::kOffStat);
+    const uint32_t sK = base + L::kOffK, sV = base + L::kOffV, sQ = base + L::kOffQ, sDO = base + L::kOffDO;
     volatile int* abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -162,17 +144,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->kv_full), 1);
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(smem_u32(&bars->q_full[s]), 1);
+            mbar_init(smem_u32(&bars->q_empty[s]), 1);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->qdo_full[s]), 1 + 32);  // expect_tx arrival + the warp's lse/Delta stores
-            mbar_init(smem_u32(&bars->qdo_empty[s]), 1);
+            mbar_init(smem_u32(&bars->do_full[s]), 1 + 32);          // expect_tx + the warp's lse/Delta stores
+            mbar_init(smem_u32(&bars->do_empty[s]), 1 + kCompute);   // c retired + Delta read by every thread
         }
         mbar_init(smem_u32(&bars->s_full), 1);
         mbar_init(smem_u32(&bars->dp_full), 1);
+        mbar_init(smem_u32(&bars->p_ready), kCompute);
         mbar_init(smem_u32(&bars->ds_ready), kCompute);
-        mbar_init(smem_u32(&bars->dq_full), 1);
-        mbar_init(smem_u32(&bars->dq_free), kCompute);
         mbar_init(smem_u32(&bars->acc_done), 1);
-        // the layout needs the 1024-byte alignment the declaration asks for (swizzle atoms)
+        // the swizzled layout needs the 1024-byte alignment the declaration asks for
         bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
         if (base & 1023u) atomicCAS(a.status, 0, 99);
         fence_mbar_init();
@@ -191,8 +176,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (warp == 0) {
         // ---------------------------------------------------- producer warp
-        // lane 0 issues the TMA copies; all 32 lanes stage lse (base 2) and Delta of
-        // the step's 128 query rows, so no compute thread waits on global memory.
         const float log2e = 1.4426950408889634f;
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -209,7 +192,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         StepMeta cur = load_meta(a, l0), nxt = cur;
         if (llen > 1) nxt = load_meta(a, l0 + 1);
         for (int it = 0; it < n_it; ++it) {
-            const int st = it & 1;
             const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
             if (hh == 0 && it > 0) {
                 cur = nxt;
@@ -224,16 +206,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 lv[u] = row < a.T ? __ldg(a.lse + (int64_t)h * a.T + row) * log2e : 0.f;
                 dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
             }
-            if (it >= 2) mbar_wait(smem_u32(&bars->qdo_empty[st]), ((it >> 1) - 1) & 1, abort, a.status, 11);
-            const uint32_t f = smem_u32(&bars->qdo_full[st]);
+            const int qs = it % 3, ds = it & 1;
+            if (it >= 3) mbar_wait(smem_u32(&bars->q_empty[qs]), ((it / 3) - 1) & 1, abort, a.status, 21);
             if (lane == 0) {
-                mbar_arrive_expect_tx(f, 2 * kTile);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, f, c * 64, h, row0);
-                    tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
-                }
+                const uint32_t f = smem_u32(&bars->q_full[qs]);
+                mbar_arrive_expect_tx(f, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + qs * kTile + c * kBox, f, c * 64, h, row0);
             }
-            float* stat = s_stat + st * 256;
+            if (it >= 2) mbar_wait(smem_u32(&bars->do_empty[ds]), ((it >> 1) - 1) & 1, abort, a.status, 22);
+            const uint32_t f = smem_u32(&bars->do_full[ds]);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(f, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + ds * kTile + c * kBox, f, c * 64, h, row0);
+            }
+            float* stat = s_stat + ds * 256;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 stat[lane + 32 * u] = lv[u];
@@ -246,9 +232,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
             constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);   // A TMEM, B MN-major
-            constexpr uint32_t idMM = idesc_bf16_f32(128, 128, true, true);    // A, B MN-major
-            auto issue_s = [&](int st) {  // a: S^T = K Q^T -> A
-                const uint32_t q = sQ + st * kTile;
+            auto issue_s = [&](int it) {  // a: S^T = K Q^T -> A
+                const int qs = it % 3;
+                mbar_wait(smem_u32(&bars->q_full[qs]), (it / 3) & 1, abort, a.status, 23);
+                tc_fence_after();
+                const uint32_t q = sQ + qs * kTile;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
@@ -256,8 +244,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 }
                 mma_commit(smem_u32(&bars->s_full));
             };
-            auto issue_dp = [&](int st) {  // b: dP^T = V dO^T -> B
-                const uint32_t d = sDO + st * kTile;
+            auto issue_dp = [&](int it) {  // b: dP^T = V dO^T -> B
+                const int ds = it & 1;
+                mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 24);
+                tc_fence_after();
+                const uint32_t d = sDO + ds * kTile;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
@@ -265,39 +256,32 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 }
                 mma_commit(smem_u32(&bars->dp_full));
             };
-            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 12);
-            mbar_wait(smem_u32(&bars->qdo_full[0]), 0, abort, a.status, 13);
+            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 25);
             tc_fence_after();
             issue_s(0);
             issue_dp(0);
             for (int it = 0; it < n_it; ++it) {
-                const int st = it & 1;
-                const uint32_t q = sQ + st * kTile, d = sDO + st * kTile;
-                mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 15);
+                const int qs = it % 3, ds = it & 1;
+                // c: dV += P^T dO, once P^T is in A
+                mbar_wait(smem_u32(&bars->p_ready), it & 1, abort, a.status, 26);
                 tc_fence_after();
-                // c: dV += P^T dO ; d: dK += dS^T Q  (A operands from region A)
+                const uint32_t d = sDO + ds * kTile;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tDV, tA + kk * 8, smem_desc_sw128(d + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                if (it + 2 < n_it) mma_commit(smem_u32(&bars->do_empty[ds]));
+                // a of the next step: A is rewritten only after c has read it (issue order)
+                if (it + 1 < n_it) issue_s(it + 1);
+                // d: dK += dS^T Q, once dS^T is in B
+                mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 27);
+                tc_fence_after();
+                const uint32_t q = sQ + qs * kTile;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDK, tA + 64 + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
-                // e: dQp = dS K -> B (dP^T there was consumed before ds_ready)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tB, smem_desc_sw128(sDS + kk * 2048, kBox, 1024), smem_desc_sw128(sK + kk * 2048, kBox, 1024),
-                           idMM, kk > 0);
-                mma_commit(smem_u32(&bars->dq_full));
-                if (it + 2 < n_it) mma_commit(smem_u32(&bars->qdo_empty[st]));
-                if (it + 1 < n_it) {
-                    const int sn = (it + 1) & 1;
-                    mbar_wait(smem_u32(&bars->qdo_full[sn]), ((it + 1) >> 1) & 1, abort, a.status, 13);
-                    tc_fence_after();
-                    issue_s(sn);  // region A is rewritten only after c and d have read it (issue order)
-                    mbar_wait(smem_u32(&bars->dq_free), it & 1, abort, a.status, 14);
-                    tc_fence_after();
-                    issue_dp(sn);
-                }
+                    mma_ts(tDK, tB + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                if (it + 3 < n_it) mma_commit(smem_u32(&bars->q_empty[qs]));
+                // b of the next step: B is rewritten only after d has read it (issue order)
+                if (it + 1 < n_it) issue_dp(it + 1);
             }
             mma_commit(smem_u32(&bars->acc_done));
         }
@@ -306,24 +290,21 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int ct = threadIdx.x - 64;         // 0..255
         const int hf = ct >> 7;                  // column half
         const int wq = warp & 3;
-        const int r = wq * 32 + lane;            // TMEM lane: key row (phases 1-2), query row (dQ)
+        const int r = wq * 32 + lane;            // TMEM lane = key row
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale_log2;
-        const int kbrk_t = KT[5], kjump_t = KT[6];
-        const int kpos_r = KT[4] + r + (r >= kbrk_t ? kjump_t : 0);
+        const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
         StepMeta cur = load_meta(a, l0), nxt = cur;
         if (llen > 1) nxt = load_meta(a, l0 + 1);
         for (int it = 0; it < n_it; ++it) {
-            const int st = it & 1;
-            const int pos = it / group, hh = it - pos * group;       // query tiles outer, heads inner
+            const int ds = it & 1;
+            const int pos = it / group, hh = it - pos * group;
             if (hh == 0 && it > 0) {
                 cur = nxt;
                 if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
             }
-            const int h = g * group + hh;
-            const int row0 = cur.row0, m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
-
-            // visible query columns of this key row: a suffix [lo, m) of the tile
+            const int m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
+            // visible query columns of this key row: a suffix [lo, hi) of the tile
             int lo = 0, hi = m;
             if (r >= cur.nvalid) hi = 0;
             else if (cur.cls != 2) {
@@ -335,11 +316,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     lo = (kpos_r <= p1) ? n1 : min(m, n1 + (kpos_r - p1));
                 }
             }
-            const float* stat = s_stat + st * 256;
+            const float* stat = s_stat + ds * 256;
 
             // ---- phase 1: P^T = exp(S^T - lse) on this thread's 64 query columns
-            mbar_wait(smem_u32(&bars->qdo_full[st]), (it >> 1) & 1, abort, a.status, 16);  // lse/Delta staged
-            mbar_wait(smem_u32(&bars->s_full), it & 1, abort, a.status, 16);
+            mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 28);  // lse/Delta staged
+            mbar_wait(smem_u32(&bars->s_full), it & 1, abort, a.status, 29);
             tc_fence_after();
             float p[64];
 #pragma unroll
@@ -360,16 +341,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     }
                 }
             }
-            named_bar_sync(1, kCompute);  // every S^T read of region A is done before P^T overwrites it
+            named_bar_sync(1, kCompute);  // all S^T reads of A are done before P^T overwrites it
             {
                 uint32_t pk[32];
 #pragma unroll
                 for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(p[2 * t], p[2 * t + 1]);
                 tmem_st32(tA + lane_addr + hf * 32, pk);
             }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_ready));
 
             // ---- phase 2: dS^T = P^T (dP^T - Delta)
-            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 17);
+            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 30);
             tc_fence_after();
             uint32_t dk[32];
 #pragma unroll
@@ -382,48 +366,22 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 for (int t = 0; t < 32; t += 4) {
                     const float4 d4 = *reinterpret_cast<const float4*>(stat + 128 + c0 + t);
                     const float dq4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float ds[4];
+                    float dsv[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) ds[u] = p[ch * 32 + t + u] * (__uint_as_float(dpv[t + u]) - dq4[u]);
-                    dk[ch * 16 + t / 2] = pack_bf16x2(ds[0], ds[1]);
-                    dk[ch * 16 + t / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                    for (int u = 0; u < 4; ++u) dsv[u] = p[ch * 32 + t + u] * (__uint_as_float(dpv[t + u]) - dq4[u]);
+                    dk[ch * 16 + t / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                    dk[ch * 16 + t / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
                 }
             }
-            tmem_st32(tA + lane_addr + 64 + hf * 32, dk);
-            // dS (query-major for the dQ product): rows = key r, 128-byte swizzled
-            {
-                const uint32_t rowb = sDS + hf * kBox + r * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(rowb + ((c ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-            }
+            mbar_arrive(smem_u32(&bars->do_empty[ds]));  // Delta of this stage read
+            named_bar_sync(1, kCompute);  // all dP^T reads of B are done before dS^T overwrites it
+            tmem_st32(tB + lane_addr + hf * 32, dk);
             tmem_wait_st();
-            fence_async_smem();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->ds_ready));
-
-            // ---- dQp rows (TMEM lane = query row r) into the fp32 dQ
-            mbar_wait(smem_u32(&bars->dq_full), it & 1, abort, a.status, 18);
-            tc_fence_after();
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t q[32];
-                const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(tB + lane_addr + c0, q);
-                tmem_wait_ld();
-                if (r < m) {
-                    float* dst = a.dq_acc + ((int64_t)(row0 + r) * a.hq + h) * kD + c0;
-#pragma unroll
-                    for (int t = 0; t < 32; t += 4)
-                        red_add_v4(dst + t, __uint_as_float(q[t]) * a.scale, __uint_as_float(q[t + 1]) * a.scale,
-                                   __uint_as_float(q[t + 2]) * a.scale, __uint_as_float(q[t + 3]) * a.scale);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->dq_free));
         }
         // ---------------------------------------------------- dK, dV epilogue
-        mbar_wait(smem_u32(&bars->acc_done), 0, abort, a.status, 19);
+        mbar_wait(smem_u32(&bars->acc_done), 0, abort, a.status, 31);
         tc_fence_after();
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
@@ -452,25 +410,252 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ================================================================ dQ
+struct DqLayout {
+    static constexpr int kKStages = 3, kVStages = 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffDO = kOffQ + kTile;
+    static constexpr int kOffK = kOffDO + kTile;
+    static constexpr int kOffV = kOffK + kKStages * kTile;
+    static constexpr int kOffBar = kOffV + kVStages * kTile;
+    static constexpr int kBytes = kOffBar + 256;
+    static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+struct DqBars {
+    uint64_t qdo_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full, dp_free, ds_ready, dq_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
+    using L = DqLayout;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    DqBars* bars = reinterpret_cast<DqBars*>(smem_raw + L::kOffBar);
+    const uint32_t sQ = base + L::kOffQ, sDO = base + L::kOffDO, sK = base + L::kOffK, sV = base + L::kOffV;
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x;
+    const int qt = a.lpt[item / a.hq];
+    const int h = item % a.hq;
+    const int g = h / (a.hq / a.hkv);
+    const int* QT = a.qtiles + (size_t)qt * 12;
+    const int row0 = QT[2], m = QT[3], qpos0 = QT[4], qbrk = QT[5], qjump = QT[6];
+    const int nk = QT[8], e0 = QT[9];
+    const int* E = a.entries + (size_t)e0 * 8;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->qdo_full), 1);
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(smem_u32(&bars->k_full[s]), 1);
+            mbar_init(smem_u32(&bars->k_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&bars->v_full[s]), 1);
+            mbar_init(smem_u32(&bars->v_empty[s]), 1);
+            mbar_init(smem_u32(&bars->s_full[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->dp_full), 1);
+        mbar_init(smem_u32(&bars->dp_free), kCompute);
+        mbar_init(smem_u32(&bars->ds_ready), kCompute);
+        mbar_init(smem_u32(&bars->dq_done), 1);
+        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
+        if (base & 1023u) atomicCAS(a.status, 0, 99);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (bars->abort) return;
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t tS = tmem, tDP = tmem + 256, tDQ = tmem + 384;   // S0 [0,128), S1 [128,256)
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            const uint32_t f = smem_u32(&bars->qdo_full);
+            mbar_arrive_expect_tx(f, 2 * kTile);
+            for (int c = 0; c < 2; ++c) {
+                tma_load_3d(&tmQ, sQ + c * kBox, f, c * 64, h, row0);
+                tma_load_3d(&tmDO, sDO + c * kBox, f, c * 64, h, row0);
+            }
+            int k0_next = nk > 0 ? __ldg(E) : 0;
+            for (int j = 0; j < nk; ++j) {
+                const int k0 = k0_next;
+                if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
+                const int ks = j % 3, vs = j & 1;
+                if (j >= 3) mbar_wait(smem_u32(&bars->k_empty[ks]), ((j / 3) - 1) & 1, abort, a.status, 41);
+                const uint32_t kf = smem_u32(&bars->k_full[ks]);
+                mbar_arrive_expect_tx(kf, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmK, sK + ks * kTile + c * kBox, kf, c * 64, g, k0);
+                if (j >= 2) mbar_wait(smem_u32(&bars->v_empty[vs]), ((j >> 1) - 1) & 1, abort, a.status, 42);
+                const uint32_t vf = smem_u32(&bars->v_full[vs]);
+                mbar_arrive_expect_tx(vf, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmV, sV + vs * kTile + c * kBox, vf, c * 64, g, k0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);
+            mbar_wait(smem_u32(&bars->qdo_full), 0, abort, a.status, 43);
+            tc_fence_after();
+            for (int j = 0; j <= nk; ++j) {
+                if (j < nk) {
+                    const int ks = j % 3, vs = j & 1, b = j & 1;
+                    // S_j = Q K_j^T into S buffer b (it held dS_{j-2}, consumed by dQ_{j-2} issued earlier)
+                    mbar_wait(smem_u32(&bars->k_full[ks]), (j / 3) & 1, abort, a.status, 44);
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                        mma_ss(tS + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
+                               smem_desc_sw128(sK + ks * kTile + off, 16, 1024), idKK, kk > 0);
+                    }
+                    mma_commit(smem_u32(&bars->s_full[b]));
+                    // dP_j = dO V_j^T, once dP_{j-1} has been read
+                    mbar_wait(smem_u32(&bars->v_full[vs]), (j >> 1) & 1, abort, a.status, 45);
+                    if (j >= 1) mbar_wait(smem_u32(&bars->dp_free), (j - 1) & 1, abort, a.status, 46);
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                        mma_ss(tDP, smem_desc_sw128(sDO + off, 16, 1024),
+                               smem_desc_sw128(sV + vs * kTile + off, 16, 1024), idKK, kk > 0);
+                    }
+                    mma_commit(smem_u32(&bars->dp_full));
+                    if (j + 2 < nk) mma_commit(smem_u32(&bars->v_empty[vs]));
+                }
+                if (j >= 1) {
+                    // dQ += dS_{j-1} K_{j-1}, dS from TMEM
+                    const int jj = j - 1, ks = jj % 3, b = jj & 1;
+                    mbar_wait(smem_u32(&bars->ds_ready), jj & 1, abort, a.status, 47);
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tDQ, tS + b * 128 + kk * 8, smem_desc_sw128(sK + ks * kTile + kk * 2048, kBox, 1024),
+                               idTM, (jj > 0 || kk > 0));
+                    if (jj + 3 < nk) mma_commit(smem_u32(&bars->k_empty[ks]));
+                }
+            }
+            mma_commit(smem_u32(&bars->dq_done));
+        }
+    } else {
+        // ---------------------------------------------------- compute warpgroups
+        const int ct = threadIdx.x - 64;
+        const int hf = ct >> 7;                  // key-column half
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;            // TMEM lane = query row
+        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const float sl2 = a.scale_log2;
+        const int qpos = qpos0 + r + (r >= qbrk ? qjump : 0);
+        const int64_t grow = (int64_t)row0 + r;
+        const float lse2 = grow < a.T ? __ldg(a.lse + (int64_t)h * a.T + grow) * 1.4426950408889634f : 0.f;
+        const float delta = grow < a.T ? __ldg(a.delta + (int64_t)h * a.T + grow) : 0.f;
+        int4 e_lo = make_int4(0, 0, 0, 0), e_hi = make_int4(0, 0, 0, 0);
+        if (nk > 0) {
+            e_lo = __ldg(reinterpret_cast<const int4*>(E));
+            e_hi = __ldg(reinterpret_cast<const int4*>(E) + 1);
+        }
+        for (int j = 0; j < nk; ++j) {
+            const int b = j & 1;
+            const int4 c_lo = e_lo, c_hi = e_hi;
+            if (j + 1 < nk) {
+                e_lo = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
+                e_hi = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8) + 1);
+            }
+            // record: k0, nvalid, kpos0, kbrk | kjump, cls, ktile, key_rank
+            int cnt = (r < m) ? c_lo.y : 0;
+            if (r < m && c_hi.y != 2) cnt = visible_keys(qpos, c_lo.y, c_lo.z, c_lo.w, c_hi.x);
+            mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 48);
+            mbar_wait(smem_u32(&bars->dp_full), j & 1, abort, a.status, 49);
+            tc_fence_after();
+            uint32_t sv[2][32], dpv[2][32];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                tmem_ld32(tS + b * 128 + lane_addr + hf * 64 + ch * 32, sv[ch]);
+                tmem_ld32(tDP + lane_addr + hf * 64 + ch * 32, dpv[ch]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->dp_free));
+            uint32_t pk[32];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int t = 0; t < 32; t += 2) {
+                    const int i = hf * 64 + ch * 32 + t;
+                    float p0 = ex2(fmaf(__uint_as_float(sv[ch][t]), sl2, -lse2));
+                    float p1 = ex2(fmaf(__uint_as_float(sv[ch][t + 1]), sl2, -lse2));
+                    p0 = i < cnt ? p0 : 0.f;
+                    p1 = i + 1 < cnt ? p1 : 0.f;
+                    pk[ch * 16 + t / 2] = pack_bf16x2(p0 * (__uint_as_float(dpv[ch][t]) - delta),
+                                                      p1 * (__uint_as_float(dpv[ch][t + 1]) - delta));
+                }
+            named_bar_sync(1, kCompute);  // all S reads of buffer b are done before dS overwrites it
+            tmem_st32(tS + b * 128 + lane_addr + hf * 32, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->ds_ready));
+        }
+        // ---------------------------------------------------- dQ epilogue
+        mbar_wait(smem_u32(&bars->dq_done), 0, abort, a.status, 50);
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            uint32_t v[32];
+            const int c0 = hf * 64 + ch * 32;
+            tmem_ld32(tDQ + lane_addr + c0, v);
+            tmem_wait_ld();
+            if (r < m) {
+                float4* dst = reinterpret_cast<float4*>(a.dq_acc + ((int64_t)(row0 + r) * a.hq + h) * kD + c0);
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    dst[t] = make_float4(__uint_as_float(v[4 * t]) * a.scale, __uint_as_float(v[4 * t + 1]) * a.scale,
+                                         __uint_as_float(v[4 * t + 2]) * a.scale,
+                                         __uint_as_float(v[4 * t + 3]) * a.scale);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 }  // namespace
 
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_ktiles, int num_sms, cudaStream_t stream) {
+                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
     static bool configured = false;
     if (!configured) {
-        if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdLayout::kDynSmem) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvLayout::kBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqLayout::kBytes) !=
+                cudaSuccess)
             return -1;
         configured = true;
     }
-    const int64_t rows = a.T * a.hq;
-    const int64_t dq_vec4 = a.T * a.hq * kD / 4;
-    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, reinterpret_cast<float4*>(a.dq_acc),
-                                                     rows, a.hq, a.T, dq_vec4);
+    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
-    const int64_t ctas = (int64_t)n_ktiles * a.hkv;
-    bwd_kernel<<<(unsigned)ctas, kThreads, BwdLayout::kDynSmem, stream>>>(q, k, v, dout, a);
+    dkdv_kernel<<<(unsigned)((int64_t)n_tiles * a.hkv), kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    dq_kernel<<<(unsigned)((int64_t)n_tiles * a.hq), kThreads, DqLayout::kBytes, stream>>>(q, k, v, dout, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -48,6 +48,7 @@ int launch_fwd_f32(int dqk, int dv, const FwdF32Args& a, int n_items, cudaStream
 struct BwdArgs {
     const int32_t* qtiles;
     const int32_t* entries;
+    const int32_t* lpt;
     const int32_t* kt_off;
     const int32_t* kt_list;
     const int32_t* kt_lpt;
@@ -55,7 +56,7 @@ struct BwdArgs {
     const __nv_bfloat16* dout;
     const float* lse;
     float* delta;   // [hq, T] workspace
-    float* dq_acc;  // [T, hq, dqk] fp32 workspace / output
+    float* dq_acc;  // [T, hq, dqk] fp32 output
     float* dk;      // [T, hkv, dqk]
     float* dv;      // [T, hkv, dv]
     int32_t hq, hkv;
@@ -65,6 +66,6 @@ struct BwdArgs {
     int* status;
 };
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_ktiles, int num_sms, cudaStream_t stream);
+                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream);
 
 }  // namespace thd
