@@ -8,16 +8,20 @@
 // causal attention with EOD reset.
 //
 // One CTA computes one (query tile, query head) work item, items taken in
-// longest-first order.  Warp roles (192 threads):
-//   warp 0      TMA producer: Q tile once, then K and V of every listed entry
-//               into a two-stage ring (128-byte swizzled boxes of 64 columns).
+// longest-first order.  Warp roles (352 threads):
+//   warp 0      TMA producer of the Q tile and of K of every listed entry;
+//   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
+//               boxes of 64 columns).
 //   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
-//               score buffers, then O += P_{j-1} V_{j-1} with P read from TMEM.
-//   warps 2-5   softmax warpgroup, one query row per thread: reads S_j from TMEM,
-//               masks PARTIAL entries only, keeps the running max / sum in fp32
-//               (base-2, scale folded in), writes P_j as bf16 over S_j, and
-//               rescales O in TMEM only when the running max grows by more than
-//               2^8 (lazy correction); finally O / l and lse to global memory.
+//               score buffers, running two tiles ahead of O += P_j V_j (P read
+//               from TMEM).
+//   warps 3-10  two softmax warpgroups; a thread owns half of one query row: it
+//               reads its 64 columns of S_j from TMEM, masks PARTIAL entries only,
+//               keeps the running max / sum in fp32 (base-2, scale folded in; the
+//               two halves' maxima meet in shared memory once per tile), writes its
+//               P_j columns as bf16 over S_j, and rescales its half of O in TMEM only
+//               when the running max grows by more than 2^8 (lazy correction);
+//               finally O / l and lse to global memory.
 // TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,256+DV) O.
 #include <cuda_bf16.h>
 
@@ -28,31 +32,34 @@ namespace thd {
 namespace {
 
 constexpr int BM = 128, BN = 128, kMaxStages = 3;
-constexpr int kThreads = 192;
+constexpr int kSoftmax = 256;          // two softmax warpgroups
+constexpr int kThreads = 96 + kSoftmax;  // K producer, MMA issuer, V producer, softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int DQK, int DV>
 struct FwdLayout {
-    // K/V ring depth: a stage is held from its load until its PV product retires, so
-    // three stages keep one load in flight ahead of the two tiles in use (D=128);
-    // the 192-wide keys of expanded MLA leave room for two.
-    static constexpr int NST = (DQK + DV <= 256) ? 3 : 2;
+    // Separate K and V rings: K_j is released as soon as S_j retires, V_j once PV_j
+    // has; each ring has its own producer warp, so neither load waits on the other.
+    static constexpr int NK = (DQK <= 128) ? 3 : 2;
+    static constexpr int NV = (DQK <= 128) ? 3 : 2;
     static constexpr int kBox = BM * 128;  // one 64-column, 128-row swizzled box: 16 KB
     static constexpr int kQBytes = BM * DQK * 2;
     static constexpr int kKBytes = BN * DQK * 2;
     static constexpr int kVBytes = BN * DV * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + NST * kKBytes;
-    static constexpr int kOffBar = kOffV + NST * kVBytes;
-    static constexpr int kBytes = kOffBar + 256;
-    static constexpr int kDynSmem = kBytes + 1024;  // slack for 1024-byte alignment
+    static constexpr int kOffV = kOffK + NK * kKBytes;
+    static constexpr int kOffBar = kOffV + NV * kVBytes;
+    static constexpr int kOffXchg = kOffBar + 256;          // [2 buffers][2 halves][128 rows] fp32
+    static constexpr int kBytes = kOffXchg + 2 * 2 * 128 * 4;
+    static constexpr int kDynSmem = kBytes;                 // base is 1024-aligned by declaration (checked)
     static_assert(kDynSmem <= 232448, "shared memory budget");
 };
 
 struct Bars {
-    uint64_t q_full, k_full[kMaxStages], v_full[kMaxStages], kv_empty[kMaxStages], s_full[2], p_full[2], o_done;
+    uint64_t q_full, k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages], s_full[2],
+        p_full[2], o_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -60,6 +67,10 @@ struct Bars {
 // Number of leading key columns of an entry visible to a query at global position
 // qpos: key t sits at kpos0 + t + (t >= kbrk ? kjump : 0), positions increase with
 // t, so the visible keys are a prefix of the nvalid listed ones.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ int visible_prefix(int qpos, int nvalid, int kpos0, int kbrk, int kjump) {
     if (qpos < kpos0) return 0;
     const int a = min(kbrk, qpos - kpos0 + 1);
@@ -74,11 +85,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
     using L = FwdLayout<DQK, DV>;
-    constexpr int NST = L::NST;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    Bars* bars = reinterpret_cast<Bars*>(smem_raw + (base - raw) + L::kOffBar);
+    constexpr int NK = L::NK, NV = L::NV;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    Bars* bars = reinterpret_cast<Bars*>(smem_raw + L::kOffBar);
+    float* xch = reinterpret_cast<float*>(smem_raw + L::kOffXchg);
     const uint32_t sQ = base + L::kOffQ, sK = base + L::kOffK, sV = base + L::kOffV;
     volatile int* abort = &bars->abort;
 
@@ -94,17 +105,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < NK; ++s) {
             mbar_init(smem_u32(&bars->k_full[s]), 1);
+            mbar_init(smem_u32(&bars->k_empty[s]), 1);
+        }
+        for (int s = 0; s < NV; ++s) {
             mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+            mbar_init(smem_u32(&bars->v_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&bars->s_full[b]), 1);
-            mbar_init(smem_u32(&bars->p_full[b]), 128);
+            mbar_init(smem_u32(&bars->p_full[b]), kSoftmax);
         }
         mbar_init(smem_u32(&bars->o_done), 1);
-        bars->abort = *reinterpret_cast<volatile int*>(a.status);
+        // the swizzled layout needs the 1024-byte alignment the declaration asks for
+        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
+        if (base & 1023u) atomicCAS(a.status, 0, 99);
         fence_mbar_init();
     }
     __syncthreads();
@@ -118,68 +134,88 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 2) {
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            const uint32_t qf = smem_u32(&bars->q_full);
-            mbar_arrive_expect_tx(qf, L::kQBytes);
-            for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
+            // ------------------------------------------------ TMA producers: warp 0 Q and K, warp 2 V
+            const bool is_k = warp == 0;
+            if (is_k) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                const uint32_t qf = smem_u32(&bars->q_full);
+                mbar_arrive_expect_tx(qf, L::kQBytes);
+                for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
+            } else {
+                tma_prefetch_desc(&tmV);
+            }
+            const int ns = is_k ? NK : NV;
             int k0_next = nk > 0 ? __ldg(E) : 0;
             for (int j = 0; j < nk; ++j) {
-                const int st = j % NST;
+                const int st = j % ns;
                 const int k0 = k0_next;
                 if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
-                if (j >= NST) mbar_wait(smem_u32(&bars->kv_empty[st]), ((j / NST) - 1) & 1, abort, a.status, 1);
-                const uint32_t kf = smem_u32(&bars->k_full[st]), vf = smem_u32(&bars->v_full[st]);
-                mbar_arrive_expect_tx(kf, L::kKBytes);
-                for (int c = 0; c < DQK / 64; ++c)
-                    tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
-                mbar_arrive_expect_tx(vf, L::kVBytes);
-                for (int c = 0; c < DV / 64; ++c)
-                    tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, k0);
+                if (is_k) {
+                    if (j >= NK) mbar_wait(smem_u32(&bars->k_empty[st]), ((j / NK) - 1) & 1, abort, a.status, 1);
+                    const uint32_t kf = smem_u32(&bars->k_full[st]);
+                    mbar_arrive_expect_tx(kf, L::kKBytes);
+                    for (int c = 0; c < DQK / 64; ++c)
+                        tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
+                } else {
+                    if (j >= NV) mbar_wait(smem_u32(&bars->v_empty[st]), ((j / NV) - 1) & 1, abort, a.status, 9);
+                    const uint32_t vf = smem_u32(&bars->v_full[st]);
+                    mbar_arrive_expect_tx(vf, L::kVBytes);
+                    for (int c = 0; c < DV / 64; ++c)
+                        tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, k0);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
+            // Order: S_0, S_1, then per tile PV_j followed by S_{j+2}; S_{j+2} reuses the
+            // TMEM buffer of S_j / P_j only after PV_j (issue order), and PV_j is never
+            // queued behind a score tile that is still waiting for its keys.
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
+            auto issue_s = [&](int j) {
+                const int st = j % NK, b = j & 1;
+                mbar_wait(smem_u32(&bars->k_full[st]), (j / NK) & 1, abort, a.status, 3);
+                tc_fence_after();
+                const uint32_t kb = sK + st * L::kKBytes;
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
+                    mma_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                           idS, kk > 0);
+                }
+                mma_commit(smem_u32(&bars->s_full[b]));
+                if (j + NK < nk) mma_commit(smem_u32(&bars->k_empty[st]));
+            };
             mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
             tc_fence_after();
-            for (int j = 0; j <= nk; ++j) {
-                if (j < nk) {
-                    const int st = j % NST, b = j & 1;
-                    mbar_wait(smem_u32(&bars->k_full[st]), (j / NST) & 1, abort, a.status, 3);
-                    tc_fence_after();
-                    const uint32_t kb = sK + st * L::kKBytes;
+            if (nk > 0) issue_s(0);
+            if (nk > 1) issue_s(1);
+            for (int j = 0; j < nk; ++j) {
+                const int st = j % NV, b = j & 1;
+                mbar_wait(smem_u32(&bars->p_full[b]), (j >> 1) & 1, abort, a.status, 4);
+                mbar_wait(smem_u32(&bars->v_full[st]), (j / NV) & 1, abort, a.status, 5);
+                tc_fence_after();
+                const uint32_t vb = sV + st * L::kVBytes;
 #pragma unroll
-                    for (int kk = 0; kk < DQK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-                        mma_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
-                               smem_desc_sw128(kb + off, 16, 1024), idS, kk > 0);
-                    }
-                    mma_commit(smem_u32(&bars->s_full[b]));
-                }
-                if (j >= 1) {
-                    const int jj = j - 1, st = jj % NST, b = jj & 1;
-                    mbar_wait(smem_u32(&bars->p_full[b]), (jj >> 1) & 1, abort, a.status, 4);
-                    mbar_wait(smem_u32(&bars->v_full[st]), (jj / NST) & 1, abort, a.status, 5);
-                    tc_fence_after();
-                    const uint32_t vb = sV + st * L::kVBytes;
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tmem + 256, tmem + b * 128 + kk * 8,
-                               smem_desc_sw128(vb + kk * 2048, L::kBox, 1024), idPV, (jj > 0 || kk > 0));
-                    mma_commit(smem_u32(&bars->o_done));
-                    if (jj + NST < nk) mma_commit(smem_u32(&bars->kv_empty[st]));  // producer reuses stage
-                }
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(tmem + 256, tmem + b * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, L::kBox, 1024), idPV,
+                           (j > 0 || kk > 0));
+                mma_commit(smem_u32(&bars->o_done));
+                if (j + NV < nk) mma_commit(smem_u32(&bars->v_empty[st]));
+                if (j + 2 < nk) issue_s(j + 2);
             }
         }
     } else {
-        // ---------------------------------------------------- softmax warpgroup
+        // ---------------------------------------------------- softmax warpgroups
+        // Two warpgroups; thread (row, half) owns 64 of the row's 128 score columns
+        // and DV/2 of its output columns.  Row maxima are combined through shared
+        // memory once per tile (double-buffered); row sums once at the end.
+        const int ct = threadIdx.x - 96;
+        const int hf = ct >> 7;
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
@@ -203,28 +239,32 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int nvalid = c_lo.y;
             int cnt = nvalid;
             if (c_hi.y != 2) cnt = visible_prefix(qpos, nvalid, c_lo.z, c_lo.w, c_hi.x);
+            cnt -= hf * 64;  // visible columns within this thread's half
             mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 6);
             tc_fence_after();
 
-            uint32_t sr[4][32];
+            uint32_t sr[2][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + b * 128 + c * 32, sr[c]);
+            for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_addr + b * 128 + hf * 64 + c * 32, sr[c]);
             tmem_wait_ld();
-            // masked scores -> -inf; row max with 8 independent partial maxima (raw units)
+            // masked scores -> -inf; partial row max with 8 independent maxima (raw units)
             float pm[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
                     float v = __uint_as_float(sr[c][t]);
-                    if (cnt < 128) v = (c * 32 + t < cnt) ? v : -INFINITY;
+                    if (cnt < 64) v = (c * 32 + t < cnt) ? v : -INFINITY;
                     sr[c][t] = __float_as_uint(v);
                     pm[t & 7] = fmaxf(pm[t & 7], v);
                 }
-            const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sl2;
+            const float pmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            xch[(b * 2 + hf) * 128 + row] = pmax;
+            named_bar_sync(1, kSoftmax);  // both halves' scores are read and their maxima posted
+            const float mx = fmaxf(pmax, xch[(b * 2 + (hf ^ 1)) * 128 + row]) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + kRescaleThreshold;
             const float m_use = grow ? m_new : m_run;
@@ -233,20 +273,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             float ps[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            {
                 uint32_t pk[32];
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
-                        const int c = half * 2 + c2;
                         const float p0 = ex2(fmaf(__uint_as_float(sr[c][t]), sl2, -m_safe));
                         const float p1 = ex2(fmaf(__uint_as_float(sr[c][t + 1]), sl2, -m_safe));
                         ps[(t >> 1) & 7] += p0 + p1;
-                        pk[c2 * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
+                        pk[c * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
                     }
-                tmem_st32(tmem + lane_addr + b * 128 + half * 32, pk);
+                tmem_st32(tmem + lane_addr + b * 128 + hf * 32, pk);  // P as bf16 over S
             }
             const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l_run = l_run * alpha + sum;
@@ -257,13 +295,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-                    for (int c = 0; c < DV / 32; ++c) {
+                    for (int c = 0; c < DV / 64; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+                        const uint32_t col = 256 + hf * (DV / 2) + c * 32;
+                        tmem_ld32(tmem + lane_addr + col, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                        tmem_st32(tmem + lane_addr + 256 + c * 32, o);
+                        tmem_st32(tmem + lane_addr + col, o);
                     }
                 }
             }
@@ -274,12 +313,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // ---------------------------------------------------- epilogue
         if (nk > 0) mbar_wait(smem_u32(&bars->o_done), (nk - 1) & 1, abort, a.status, 8);
         tc_fence_after();
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-        __nv_bfloat16* orow = a.o + ((size_t)(row0 + row) * a.hq + h) * DV;
+        named_bar_sync(1, kSoftmax);  // last maxima read before the buffer is reused for the sums
+        xch[hf * 128 + row] = l_run;
+        named_bar_sync(1, kSoftmax);
+        const float l_tot = l_run + xch[(hf ^ 1) * 128 + row];
+        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        __nv_bfloat16* orow = a.o + ((size_t)(row0 + row) * a.hq + h) * DV + hf * (DV / 2);
 #pragma unroll
-        for (int c = 0; c < DV / 32; ++c) {
+        for (int c = 0; c < DV / 64; ++c) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + 256 + c * 32, o);
+            tmem_ld32(tmem + lane_addr + 256 + hf * (DV / 2) + c * 32, o);
             tmem_wait_ld();
             uint32_t pk[16];
 #pragma unroll
@@ -291,7 +334,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
         }
-        if (row < m) a.lse[(size_t)h * a.T + row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+        if (row < m && hf == 0)
+            a.lse[(size_t)h * a.T + row0 + row] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
     }
     tc_fence_before();
     __syncthreads();

@@ -57,25 +57,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete.  Gives up after kWaitTimeoutNs, or at
-// once when another thread of the CTA already gave up (*abort != 0): it then records
-// `code` in the plan's device status word and returns false, so that the kernel
-// drains and exits instead of hanging.
+// Waits for the phase of `parity` to complete.  The poll loop itself only issues
+// try_wait; every 1024 polls it also checks the CTA's abort flag, the plan's
+// device status word (set when any CTA gave up) and the elapsed time.  After
+// kWaitTimeoutNs it records `code` in the status word and returns false, so that
+// the kernel drains and exits instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* status, int code) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    uint32_t polls = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (*reinterpret_cast<volatile int*>(status) != 0) {  // another CTA already gave up
-            *abort = 1;
-            return false;
-        }
-        if (globaltimer() - t0 > kWaitTimeoutNs) {
-            *abort = 1;
-            atomicCAS(status, 0, code);
-            return false;
+        if ((++polls & 1023u) == 0) {
+            if (*abort) return false;
+            if (*reinterpret_cast<volatile int*>(status) != 0) {  // another CTA already gave up
+                *abort = 1;
+                return false;
+            }
+            if (globaltimer() - t0 > kWaitTimeoutNs) {
+                *abort = 1;
+                atomicCAS(status, 0, code);
+                return false;
+            }
         }
     }
 }
