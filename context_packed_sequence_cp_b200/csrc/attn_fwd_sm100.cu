@@ -247,18 +247,34 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_addr + b * 128 + hf * 64 + c * 32, sr[c]);
             tmem_wait_ld();
-            // masked scores -> -inf; partial row max with 8 independent maxima (raw units)
-            float pm[8];
+            if (__any_sync(0xffffffffu, cnt < 64)) {  // PARTIAL entry or short key run: mask
 #pragma unroll
-            for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if (c * 32 + t >= cnt) sr[c][t] = __float_as_uint(-INFINITY);
+            }
+            // Exponentials against the running max, with the tile's row max taken in the
+            // same pass (the max runs on the ALU while the exponentials hold the XU).
+            // Only when the max grows by more than 2^8 is the tile recomputed (rare).
+            const float m_ref = (m_run == -INFINITY) ? 0.f : m_run;
+            float pm[8], ps[8];
+            uint32_t pk[32];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                pm[u] = -INFINITY;
+                ps[u] = 0.f;
+            }
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    float v = __uint_as_float(sr[c][t]);
-                    if (cnt < 64) v = (c * 32 + t < cnt) ? v : -INFINITY;
-                    sr[c][t] = __float_as_uint(v);
-                    pm[t & 7] = fmaxf(pm[t & 7], v);
+                for (int t = 0; t < 32; t += 2) {
+                    const float s0 = __uint_as_float(sr[c][t]), s1 = __uint_as_float(sr[c][t + 1]);
+                    pm[(t >> 1) & 7] = fmaxf(pm[(t >> 1) & 7], fmaxf(s0, s1));
+                    const float p0 = ex2(fmaf(s0, sl2, -m_ref));
+                    const float p1 = ex2(fmaf(s1, sl2, -m_ref));
+                    ps[(t >> 1) & 7] += p0 + p1;
+                    pk[c * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
                 }
             const float pmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                      fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
@@ -270,22 +286,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const float m_use = grow ? m_new : m_run;
             const float m_safe = (m_use == -INFINITY) ? 0.f : m_use;
             const float alpha = grow ? ex2(m_run - m_safe) : 1.f;
-            float ps[8];
+            if (__any_sync(0xffffffffu, grow)) {  // rare: redo this row's tile against the new max
+                if (grow) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-            {
-                uint32_t pk[32];
+                    for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[c][t]), sl2, -m_safe));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[c][t + 1]), sl2, -m_safe));
-                        ps[(t >> 1) & 7] += p0 + p1;
-                        pk[c * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
-                    }
-                tmem_st32(tmem + lane_addr + b * 128 + hf * 32, pk);  // P as bf16 over S
+                        for (int t = 0; t < 32; t += 2) {
+                            const float p0 = ex2(fmaf(__uint_as_float(sr[c][t]), sl2, -m_safe));
+                            const float p1 = ex2(fmaf(__uint_as_float(sr[c][t + 1]), sl2, -m_safe));
+                            ps[(t >> 1) & 7] += p0 + p1;
+                            pk[c * 16 + (t >> 1)] = pack_bf16x2(p0, p1);
+                        }
+                }
             }
+            tmem_st32(tmem + lane_addr + b * 128 + hf * 32, pk);  // P as bf16 over S (read above)
             const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
