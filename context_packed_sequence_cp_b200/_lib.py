@@ -10,12 +10,13 @@ LIB_PATH = os.path.join(_HERE, "libthdcp.so")
 THD_OK = 0
 THD_DTYPE_BF16 = 0
 THD_DTYPE_FP32 = 1
+NOALLOC_MAX_ROWS_X_HEADS = 8388608
 QT_FIELDS = 12
 EN_FIELDS = 8
 
 ERRORS = {
     -1: "INVALID_ARG", -2: "BAD_SEQLENS", -3: "NOT_DIVISIBLE", -4: "MISALIGNED",
-    -5: "NOT_UPLOADED", -6: "CUDA", -7: "UNSUPPORTED", -8: "ALLOC",
+    -5: "NOT_UPLOADED", -6: "CUDA", -7: "UNSUPPORTED", -8: "ALLOC", -9: "TOO_LARGE",
 }
 
 # Every entry point of include/thdcp.h: name -> (restype, argtypes)
@@ -36,6 +37,8 @@ SIGNATURES = {
     "thd_cp_attn_bwd_workspace": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(ctypes.c_size_t)]),
     "thd_cp_attn_bwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                        _I32, _I32, _I32, _I32, _F, _I32, _P]),
+    "thd_cp_attn_bwd_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               _I32, _I32, _I32, _I32, _F, _I32, _P]),
     "thd_cp_device_status": (ctypes.c_int, [_P, _I32, _PI32]),
     "thd_cp_strerror": (ctypes.c_char_p, [ctypes.c_int]),
 }

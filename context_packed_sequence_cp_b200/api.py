@@ -160,3 +160,18 @@ def thd_cp_attn_bwd(plan: Plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, *, scale:
         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
         hq, hkv, dqk, dvd, float(scale), _DTYPES[q_rm.dtype], _stream(stream)))
     return dq, dk, dv
+
+
+def thd_cp_attn_bwd_noalloc(plan: Plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, *, scale: float | None = None,
+                            dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, stream=None):
+    """thd_cp_attn_bwd without a workspace, for callers that cannot allocate device
+    memory: the library keeps the per-row statistic in a fixed device array
+    (hq * T <= 8,388,608).  Outputs must be passed in (fp32, rank-major)."""
+    T, hq, dqk = q_rm.shape
+    hkv, dvd = k_rm.shape[1], v_rm.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    check("thd_cp_attn_bwd_noalloc", lib().thd_cp_attn_bwd_noalloc(
+        plan.handle, _ptr(q_rm), _ptr(k_rm), _ptr(v_rm), _ptr(o_rm), _ptr(lse_rm), _ptr(do_rm),
+        _ptr(dq), _ptr(dk), _ptr(dv), hq, hkv, dqk, dvd, float(scale), _DTYPES[q_rm.dtype], _stream(stream)))
+    return dq, dk, dv

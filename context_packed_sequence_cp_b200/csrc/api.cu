@@ -329,6 +329,7 @@ const char* thd_cp_strerror(int code) {
         case THD_ERR_CUDA: return "CUDA runtime or launch error";
         case THD_ERR_UNSUPPORTED: return "unsupported dtype / head dimension combination";
         case THD_ERR_ALLOC: return "allocation failed";
+        case THD_ERR_TOO_LARGE: return "hq * T exceeds the fixed scratch of the no-allocation backward";
         default: return "unknown error";
     }
 }

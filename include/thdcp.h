@@ -50,6 +50,7 @@ extern "C" {
 #define THD_ERR_CUDA          -6  /* a CUDA runtime call or a launch failed         */
 #define THD_ERR_UNSUPPORTED   -7  /* dtype / head-dim combination not built         */
 #define THD_ERR_ALLOC         -8  /* host or device allocation failed               */
+#define THD_ERR_TOO_LARGE     -9  /* hq * T exceeds the fixed scratch of thd_cp_attn_bwd_noalloc */
 
 /* ---- element types ----------------------------------------------------- */
 #define THD_DTYPE_BF16 0   /* bf16 inputs, fp32 accumulation, tcgen05 tensor cores */
@@ -207,6 +208,32 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
                     void* workspace, size_t workspace_bytes,
                     int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale,
                     int32_t dtype, void* stream);
+
+/*
+ * thd_cp_attn_bwd_noalloc -- thd_cp_attn_bwd for callers that cannot allocate
+ * device memory.  (The paper has no counterpart: this is a deployment variant of
+ * the same backward.)  thd_cp_attn_bwd wants a workspace for the per-row
+ * statistic Delta; a caller whose device memory is owned entirely by another
+ * allocator, or whose hot path may not call cudaMalloc (it can synchronise the
+ * device), cannot provide one.  This entry point keeps Delta in a fixed device
+ * array built into the library instead and allocates nothing itself.
+ *   Arguments, layouts, outputs and errors as thd_cp_attn_bwd, without the
+ *   workspace; the plan must already be uploaded.
+ *   Limit: hq * T <= THD_NOALLOC_MAX_ROWS_X_HEADS (8,388,608, i.e. 32 MiB of
+ *   fp32); larger problems return THD_ERR_TOO_LARGE without launching anything.
+ *   Every GPU that loads the library holds the 32 MiB array until the process
+ *   exits.  The first call on a device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any stream
+ *   capture.  All calls share the array: calls whose kernels overlap on the GPU
+ *   (e.g. on different streams) race on it and must be serialised by the caller.
+ *   The array is fully rewritten by each call before it is read.
+ */
+#define THD_NOALLOC_MAX_ROWS_X_HEADS 8388608
+int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm,
+                            const void* o_rm, const float* lse_rm, const void* do_rm,
+                            float* dq_rm, float* dk_rm, float* dv_rm,
+                            int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale,
+                            int32_t dtype, void* stream);
 
 /*
  * thd_cp_device_status -- every wait inside this library's kernels is bounded
