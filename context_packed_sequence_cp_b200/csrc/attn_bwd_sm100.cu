@@ -9,9 +9,10 @@
 //
 // Three kernels, none with atomics:
 //   bwd_prep   Delta_i = sum_d dO_id O_id per (row, head).
-//   dkdv       one CTA per (key tile, key/value head g), key tiles longest-first; it
-//              walks every query tile the plan's key-tile transpose lists (outer) and
-//              every query head of g's group (inner).  Key rows on TMEM lanes:
+//   dkdv       one CTA per (key tile, key/value head g), groups outermost and key
+//              tiles longest-first within a group; it walks every query tile the
+//              plan's key-tile transpose lists (outer, latest query position first)
+//              and every query head of g's group (inner).  Key rows on TMEM lanes:
 //                a  S^T  = K Q^T   -> TMEM A       b  dP^T = V dO^T -> TMEM B
 //                phase 1: P^T = exp(S^T - lse) -> bf16 over S^T (A)
 //                phase 2: dS^T = P^T (dP^T - Delta) -> bf16 over dP^T (B)
@@ -135,8 +136,12 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = a.hq / a.hkv;
-    const int kt = a.kt_lpt[blockIdx.x / a.hkv];
-    const int g = blockIdx.x % a.hkv;
+    // Groups outermost: the CTAs resident together serve one KV group, so they read
+    // the same query heads, and (their lists being prefixes of one order) the same
+    // query tiles at about the same time; the tiles are mostly L2 hits after the first.
+    const int n_kt = (int)(gridDim.x / (unsigned)a.hkv);
+    const int kt = a.kt_lpt[blockIdx.x % n_kt];
+    const int g = blockIdx.x / n_kt;
     const int* KT = a.qtiles + (size_t)kt * 12;  // key tiles are the plan's row tiles
     const int k0 = KT[2], kn = KT[3];
     const int l0 = a.kt_off[kt], llen = a.kt_off[kt + 1] - l0;

@@ -22,6 +22,8 @@
 
 #include <algorithm>
 #include <limits>
+#include <utility>
+#include <vector>
 
 namespace {
 
@@ -174,13 +176,35 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         for (int64_t t = 0; t < n_tiles; ++t) p->kt_off[t + 1] += p->kt_off[t];
         std::vector<int32_t> fill(p->kt_off.begin(), p->kt_off.end() - 1);
         p->kt_list.assign((size_t)ne * 2, 0);
-        for (int64_t qt = 0; qt < n_tiles; ++qt) {  // query tiles ascending -> lists sorted
+        for (int64_t qt = 0; qt < n_tiles; ++qt) {
             const int32_t* q = &p->qtiles[(size_t)qt * THD_QTILE_FIELDS];
             for (int64_t e = q[9]; e < (int64_t)q[9] + q[8]; ++e) {
                 const int32_t kt = p->entries[(size_t)e * THD_ENTRY_FIELDS + 6];
                 const int32_t at = fill[kt]++;
                 p->kt_list[(size_t)at * 2] = (int32_t)qt;
                 p->kt_list[(size_t)at * 2 + 1] = (int32_t)e;
+            }
+        }
+        // Each list in descending order of the query tile's last position (ties,
+        // which cannot occur within one document, by tile index).  A key tile sees
+        // exactly the query tiles of its document whose last position is at or past
+        // its first key, so every key tile's list is a prefix of one per-document
+        // order: key tiles walked at the same time read the same query tiles.
+        for (int64_t kt = 0; kt < n_tiles; ++kt) {
+            std::vector<std::pair<int32_t, int32_t>> run;
+            for (int64_t at = p->kt_off[kt]; at < p->kt_off[kt + 1]; ++at)
+                run.emplace_back(p->kt_list[(size_t)at * 2], p->kt_list[(size_t)at * 2 + 1]);
+            std::sort(run.begin(), run.end(), [&](const std::pair<int32_t, int32_t>& x,
+                                                  const std::pair<int32_t, int32_t>& y) {
+                const int32_t px = p->qtiles[(size_t)x.first * THD_QTILE_FIELDS + 7];
+                const int32_t py = p->qtiles[(size_t)y.first * THD_QTILE_FIELDS + 7];
+                return px != py ? px > py : x.first < y.first;
+            });
+            int64_t at = p->kt_off[kt];
+            for (const auto& pr : run) {
+                p->kt_list[(size_t)at * 2] = pr.first;
+                p->kt_list[(size_t)at * 2 + 1] = pr.second;
+                ++at;
             }
         }
         p->kt_lpt.resize(n_tiles);

@@ -116,7 +116,8 @@ int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out);
  *                THD_CLS_PARTIAL.  Fully masked slices are not listed.
  *   lpt          int32[n_qtiles]   query tiles by descending nk (ties by index)
  *   kt_off       int32[n_qtiles+1] CSR offsets of the key-tile transpose
- *   kt_list      int32[n_entries*2] (qtile, entry) per key tile, qtile ascending
+ *   kt_list      int32[n_entries*2] (qtile, entry) per key tile, by descending
+ *                qpos_max of the query tile (ties by qtile index)
  *   kt_lpt       int32[n_qtiles]   key tiles by descending list length
  */
 int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global,

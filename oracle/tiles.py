@@ -29,7 +29,8 @@ Record layouts (int32):
               nk, entry_off, doc_start, doc_end
   entry[8]  = k0 (rank-major), nvalid, kpos0, kbrk, kjump, cls, ktile, key_rank
   ktiles are the q-tiles themselves (same row slices); the backward transpose is
-  kt_off[n_tiles+1] / kt_list[n_entries][2] = (qtile, entry), q-tile ascending.
+  kt_off[n_tiles+1] / kt_list[n_entries][2] = (qtile, entry), each key tile's list
+  in descending order of the q-tile's qpos_max (ties by q-tile index).
   lpt: q-tiles by descending nk (ties by index); kt_lpt: key tiles by descending
   number of listed q-tiles (ties by index).
 
@@ -128,7 +129,9 @@ def tile_plan(cu_seqlens, cp: int) -> dict:
             lists[int(entries[e, 6])].append((qt, e))
     kt_off = np.zeros(n_tiles + 1, dtype=np.int32)
     kt_off[1:] = np.cumsum([len(x) for x in lists])
-    kt_list = np.array([p for x in lists for p in sorted(x)], dtype=np.int32).reshape(-1, 2)
+    # each key tile's list by descending last query position, then q-tile index
+    kt_list = np.array([p for x in lists for p in sorted(x, key=lambda pr: (-int(qtiles[pr[0], 7]), pr[0]))],
+                       dtype=np.int32).reshape(-1, 2)
     kt_lpt = np.array(sorted(range(n_tiles), key=lambda t: (-len(lists[t]), t)), dtype=np.int32)
 
     return dict(T=int(cu[-1]), cp=int(cp), Tl=int(cu[-1]) // cp, n_docs=n_docs,

@@ -148,7 +148,14 @@ def test_backward_transpose_and_lpt():
         seen = np.zeros(plan["entries"].shape[0], dtype=np.int64)
         for kt in range(n):
             lst = plan["kt_list"][plan["kt_off"][kt]:plan["kt_off"][kt + 1]]
-            assert np.all(np.diff(lst[:, 0]) >= 0)
+            qmax = plan["qtiles"][lst[:, 0], 7]
+            assert np.all(np.diff(qmax) < 0)   # descending last query position
+            # the list is every q-tile of the key tile's document whose last row is at or
+            # past the key tile's first key: a prefix of one per-document order
+            kpos_min = int(plan["q_idx"][plan["qtiles"][kt, 2]])
+            d = plan["qtiles"][kt, 1]
+            want = [qt for qt in range(n) if plan["qtiles"][qt, 1] == d and plan["qtiles"][qt, 7] >= kpos_min]
+            assert sorted(lst[:, 0].tolist()) == want
             for qt, e in lst:
                 assert plan["entries"][e, 6] == kt
                 assert plan["qtiles"][qt, 9] <= e < plan["qtiles"][qt, 9] + plan["qtiles"][qt, 8]
