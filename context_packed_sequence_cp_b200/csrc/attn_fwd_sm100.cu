@@ -12,9 +12,12 @@
 //   warp 0      TMA producer of the Q tile and of K of every listed entry;
 //   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
 //               boxes of 64 columns).
-//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
-//               score buffers, running two tiles ahead of O += P_j V_j (P read
-//               from TMEM).
+//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of three TMEM
+//               score buffers, running three tiles ahead of O += P_j V_j (P read
+//               from TMEM).  The MMA warp observes the release of P_j several
+//               hundred cycles after the softmax signals it (measured in place), so
+//               with three buffers that latency is off the softmax's path: S_{j+1}
+//               was issued after PV_{j-2}.
 //   warps 3-10  two softmax warpgroups; a thread owns half of one query row: it
 //               reads its 64 columns of S_j from TMEM, masks PARTIAL entries only,
 //               keeps the running max / sum in fp32 (base-2, scale folded in; the
@@ -22,7 +25,7 @@
 //               P_j columns as bf16 over S_j, and rescales its half of O in TMEM only
 //               when the running max grows by more than 2^8 (lazy correction);
 //               finally O / l and lse to global memory.
-// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,256+DV) O.
+// TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,384) S2/P2, [384,384+DV) O.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -32,6 +35,8 @@ namespace thd {
 namespace {
 
 constexpr int BM = 128, BN = 128, kMaxStages = 3;
+constexpr int kSBuf = 3;                 // S/P buffers in TMEM
+constexpr uint32_t kTmemO = kSBuf * 128; // first O column
 constexpr int kSoftmax = 256;          // two softmax warpgroups
 constexpr int kThreads = 96 + kSoftmax;  // K producer, MMA issuer, V producer, softmax
 constexpr uint32_t kTmemCols = 512;
@@ -58,8 +63,8 @@ struct FwdLayout {
 };
 
 struct Bars {
-    uint64_t q_full, k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages], s_full[2],
-        p_full[2], o_done;
+    uint64_t q_full, k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages],
+        s_full[kSBuf], p_full[kSBuf], o_done[kSBuf];
     uint32_t tmem_base;
     int abort;
 };
@@ -113,11 +118,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mbar_init(smem_u32(&bars->v_full[s]), 1);
             mbar_init(smem_u32(&bars->v_empty[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kSBuf; ++b) {
             mbar_init(smem_u32(&bars->s_full[b]), 1);
             mbar_init(smem_u32(&bars->p_full[b]), kSoftmax);
+            mbar_init(smem_u32(&bars->o_done[b]), 1);  // PV_j with j % kSBuf == b retired
         }
-        mbar_init(smem_u32(&bars->o_done), 1);
         // the swizzled layout needs the 1024-byte alignment the declaration asks for
         bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
         if (base & 1023u) atomicCAS(a.status, 0, 99);
@@ -177,7 +182,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
             auto issue_s = [&](int j) {
-                const int st = j % NK, b = j & 1;
+                const int st = j % NK, b = j % kSBuf;
                 mbar_wait(smem_u32(&bars->k_full[st]), (j / NK) & 1, abort, a.status, 3);
                 tc_fence_after();
                 const uint32_t kb = sK + st * L::kKBytes;
@@ -192,21 +197,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             };
             mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
             tc_fence_after();
-            if (nk > 0) issue_s(0);
-            if (nk > 1) issue_s(1);
+            for (int j = 0; j < kSBuf && j < nk; ++j) issue_s(j);
             for (int j = 0; j < nk; ++j) {
-                const int st = j % NV, b = j & 1;
-                mbar_wait(smem_u32(&bars->p_full[b]), (j >> 1) & 1, abort, a.status, 4);
+                const int st = j % NV, b = j % kSBuf;
+                mbar_wait(smem_u32(&bars->p_full[b]), (j / kSBuf) & 1, abort, a.status, 4);
                 mbar_wait(smem_u32(&bars->v_full[st]), (j / NV) & 1, abort, a.status, 5);
                 tc_fence_after();
                 const uint32_t vb = sV + st * L::kVBytes;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tmem + 256, tmem + b * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, L::kBox, 1024), idPV,
-                           (j > 0 || kk > 0));
-                mma_commit(smem_u32(&bars->o_done));
+                    mma_ts(tmem + kTmemO, tmem + b * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, L::kBox, 1024),
+                           idPV, (j > 0 || kk > 0));
+                mma_commit(smem_u32(&bars->o_done[b]));
                 if (j + NV < nk) mma_commit(smem_u32(&bars->v_empty[st]));
-                if (j + 2 < nk) issue_s(j + 2);
+                if (j + kSBuf < nk) issue_s(j + kSBuf);
             }
         }
     } else {
@@ -229,7 +233,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             e_hi = __ldg(reinterpret_cast<const int4*>(E) + 1);
         }
         for (int j = 0; j < nk; ++j) {
-            const int b = j & 1;
+            const int b = j % kSBuf, xb = j & 1;
             const int4 c_lo = e_lo, c_hi = e_hi;
             if (j + 1 < nk) {
                 e_lo = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
@@ -240,7 +244,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             int cnt = nvalid;
             if (c_hi.y != 2) cnt = visible_prefix(qpos, nvalid, c_lo.z, c_lo.w, c_hi.x);
             cnt -= hf * 64;  // visible columns within this thread's half
-            mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 6);
+            mbar_wait(smem_u32(&bars->s_full[b]), (j / kSBuf) & 1, abort, a.status, 6);
             tc_fence_after();
 
             uint32_t sr[2][32];
@@ -278,9 +282,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 }
             const float pmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                      fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-            xch[(b * 2 + hf) * 128 + row] = pmax;
+            xch[(xb * 2 + hf) * 128 + row] = pmax;
             named_bar_sync(1, kSoftmax);  // both halves' scores are read and their maxima posted
-            const float mx = fmaxf(pmax, xch[(b * 2 + (hf ^ 1)) * 128 + row]) * sl2;
+            const float mx = fmaxf(pmax, xch[(xb * 2 + (hf ^ 1)) * 128 + row]) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + kRescaleThreshold;
             const float m_use = grow ? m_new : m_run;
@@ -305,21 +309,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l_run = l_run * alpha + sum;
             m_run = m_use;
-            if (j >= 1) {
-                // PV_{j-1} must be complete before O is touched or PV_j is issued.
-                mbar_wait(smem_u32(&bars->o_done), (j - 1) & 1, abort, a.status, 7);
+            if (j >= 1 && __any_sync(0xffffffffu, grow)) {
+                // O is rescaled only once PV_{j-1} has retired.  The signal of S_j covers
+                // PV_{j-3} (issued before it), so o_done of PV_{j-1}'s buffer is at most
+                // one use behind and its parity identifies the phase.
+                mbar_wait(smem_u32(&bars->o_done[(j - 1) % kSBuf]), ((j - 1) / kSBuf) & 1, abort, a.status, 7);
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
-                    for (int c = 0; c < DV / 64; ++c) {
-                        uint32_t o[32];
-                        const uint32_t col = 256 + hf * (DV / 2) + c * 32;
-                        tmem_ld32(tmem + lane_addr + col, o);
-                        tmem_wait_ld();
+                for (int c = 0; c < DV / 64; ++c) {
+                    uint32_t o[32];
+                    const uint32_t col = kTmemO + hf * (DV / 2) + c * 32;
+                    tmem_ld32(tmem + lane_addr + col, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-                        tmem_st32(tmem + lane_addr + col, o);
-                    }
+                    for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+                    tmem_st32(tmem + lane_addr + col, o);
                 }
             }
             tmem_wait_st();
@@ -327,7 +331,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mbar_arrive(smem_u32(&bars->p_full[b]));
         }
         // ---------------------------------------------------- epilogue
-        if (nk > 0) mbar_wait(smem_u32(&bars->o_done), (nk - 1) & 1, abort, a.status, 8);
+        if (nk > 0)
+            mbar_wait(smem_u32(&bars->o_done[(nk - 1) % kSBuf]), ((nk - 1) / kSBuf) & 1, abort, a.status, 8);
         tc_fence_after();
         named_bar_sync(1, kSoftmax);  // last maxima read before the buffer is reused for the sums
         xch[hf * 128 + row] = l_run;
@@ -338,7 +343,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
         for (int c = 0; c < DV / 64; ++c) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + 256 + hf * (DV / 2) + c * 32, o);
+            tmem_ld32(tmem + lane_addr + kTmemO + hf * (DV / 2) + c * 32, o);
             tmem_wait_ld();
             uint32_t pk[16];
 #pragma unroll

@@ -59,7 +59,9 @@ def test_fwd_bf16_workload_sampled(cfg):
     assert np.abs(lse[heads][:, rows].T - want_l).max() <= LSE_MAX
 
 
-@pytest.mark.parametrize("hq,hkv,dqk,dv", [(4, 4, 128, 128), (8, 2, 128, 128), (4, 4, 192, 128), (6, 1, 128, 128)])
+# MHA, GQA with groups of 4, 6, 2 and 3, and expanded MLA
+@pytest.mark.parametrize("hq,hkv,dqk,dv", [(4, 4, 128, 128), (8, 2, 128, 128), (4, 4, 192, 128), (6, 1, 128, 128),
+                                           (4, 2, 128, 128), (3, 1, 128, 128)])
 @pytest.mark.parametrize("cp", [1, 2, 4, 8])
 def test_fwd_bf16_small_layouts_full(hq, hkv, dqk, dv, cp):
     """Random layouts spanning several tiles with ragged tails, every output compared."""
