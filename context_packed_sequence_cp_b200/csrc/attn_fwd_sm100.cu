@@ -13,11 +13,16 @@
 //   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
 //               boxes of 64 columns).
 //   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of three TMEM
-//               score buffers, running three tiles ahead of O += P_j V_j (P read
+//               score buffers, running two tiles ahead of O += P_j V_j (P read
 //               from TMEM).  The MMA warp observes the release of P_j several
-//               hundred cycles after the softmax signals it (measured in place), so
-//               with three buffers that latency is off the softmax's path: S_{j+1}
-//               was issued after PV_{j-2}.
+//               hundred cycles after the softmax signals it (measured in place);
+//               the spare third buffer keeps that latency off the softmax's path.
+//               Every barrier wait or commit between MMA groups lets the tensor
+//               pipe's short queue run dry (measured: ~60-140 cycles each), so
+//               the issuer waits once per tile (P_j released) and commits twice
+//               (PV_j retired, S_{j+2} written); the producers recycle their
+//               stages on those same two signals, and one softmax thread checks
+//               that V_j and K_{j+2} have landed before it releases P_j.
 //   warps 3-10  two softmax warpgroups; a thread owns half of one query row: it
 //               reads its 64 columns of S_j from TMEM, masks PARTIAL entries only,
 //               keeps the running max / sum in fp32 (base-2, scale folded in; the
@@ -63,8 +68,7 @@ struct FwdLayout {
 };
 
 struct Bars {
-    uint64_t q_full, k_full[kMaxStages], k_empty[kMaxStages], v_full[kMaxStages], v_empty[kMaxStages],
-        s_full[kSBuf], p_full[kSBuf], o_done[kSBuf];
+    uint64_t q_full, k_full[kMaxStages], v_full[kMaxStages], s_full[kSBuf], p_full[kSBuf], o_done[kSBuf];
     uint32_t tmem_base;
     int abort;
 };
@@ -110,14 +114,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        for (int s = 0; s < NK; ++s) {
-            mbar_init(smem_u32(&bars->k_full[s]), 1);
-            mbar_init(smem_u32(&bars->k_empty[s]), 1);
-        }
-        for (int s = 0; s < NV; ++s) {
-            mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->v_empty[s]), 1);
-        }
+        for (int s = 0; s < NK; ++s) mbar_init(smem_u32(&bars->k_full[s]), 1);
+        for (int s = 0; s < NV; ++s) mbar_init(smem_u32(&bars->v_full[s]), 1);
         for (int b = 0; b < kSBuf; ++b) {
             mbar_init(smem_u32(&bars->s_full[b]), 1);
             mbar_init(smem_u32(&bars->p_full[b]), kSoftmax);
@@ -158,14 +156,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const int st = j % ns;
                 const int k0 = k0_next;
                 if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
+                // A stage is refilled once the MMA that read it has retired: K_{j-NK} is
+                // read by S_{j-NK} (signalled on s_full), V_{j-NV} by PV_{j-NV} (o_done).
+                // NK, NV <= kSBuf, so the next use of either barrier needs the tile
+                // being loaded here: the awaited phase is never ambiguous.
                 if (is_k) {
-                    if (j >= NK) mbar_wait(smem_u32(&bars->k_empty[st]), ((j / NK) - 1) & 1, abort, a.status, 1);
+                    if (j >= NK)
+                        mbar_wait(smem_u32(&bars->s_full[(j - NK) % kSBuf]), ((j - NK) / kSBuf) & 1, abort, a.status, 1);
                     const uint32_t kf = smem_u32(&bars->k_full[st]);
                     mbar_arrive_expect_tx(kf, L::kKBytes);
                     for (int c = 0; c < DQK / 64; ++c)
                         tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
                 } else {
-                    if (j >= NV) mbar_wait(smem_u32(&bars->v_empty[st]), ((j / NV) - 1) & 1, abort, a.status, 9);
+                    if (j >= NV)
+                        mbar_wait(smem_u32(&bars->o_done[(j - NV) % kSBuf]), ((j - NV) / kSBuf) & 1, abort, a.status, 9);
                     const uint32_t vf = smem_u32(&bars->v_full[st]);
                     mbar_arrive_expect_tx(vf, L::kVBytes);
                     for (int c = 0; c < DV / 64; ++c)
@@ -176,15 +180,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
-            // Order: S_0, S_1, then per tile PV_j followed by S_{j+2}; S_{j+2} reuses the
-            // TMEM buffer of S_j / P_j only after PV_j (issue order), and PV_j is never
-            // queued behind a score tile that is still waiting for its keys.
+            // Order: S_0, S_1, then per tile PV_j followed by S_{j+2}.  S_{j+2} reuses the
+            // TMEM buffer of P_{j-1} after PV_{j-1} (issue order).  Inside the loop the
+            // only wait is for P_j: its release also vouches for V_j and K_{j+2}.
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
             auto issue_s = [&](int j) {
                 const int st = j % NK, b = j % kSBuf;
-                mbar_wait(smem_u32(&bars->k_full[st]), (j / NK) & 1, abort, a.status, 3);
-                tc_fence_after();
                 const uint32_t kb = sK + st * L::kKBytes;
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
@@ -193,15 +195,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                            idS, kk > 0);
                 }
                 mma_commit(smem_u32(&bars->s_full[b]));
-                if (j + NK < nk) mma_commit(smem_u32(&bars->k_empty[st]));
             };
             mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
-            tc_fence_after();
-            for (int j = 0; j < kSBuf && j < nk; ++j) issue_s(j);
+            for (int j = 0; j < 2 && j < nk; ++j) {
+                mbar_wait(smem_u32(&bars->k_full[j % NK]), (j / NK) & 1, abort, a.status, 3);
+                tc_fence_after();
+                issue_s(j);
+            }
             for (int j = 0; j < nk; ++j) {
                 const int st = j % NV, b = j % kSBuf;
                 mbar_wait(smem_u32(&bars->p_full[b]), (j / kSBuf) & 1, abort, a.status, 4);
-                mbar_wait(smem_u32(&bars->v_full[st]), (j / NV) & 1, abort, a.status, 5);
                 tc_fence_after();
                 const uint32_t vb = sV + st * L::kVBytes;
 #pragma unroll
@@ -209,8 +212,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     mma_ts(tmem + kTmemO, tmem + b * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, L::kBox, 1024),
                            idPV, (j > 0 || kk > 0));
                 mma_commit(smem_u32(&bars->o_done[b]));
-                if (j + NV < nk) mma_commit(smem_u32(&bars->v_empty[st]));
-                if (j + kSBuf < nk) issue_s(j + kSBuf);
+                if (j + 2 < nk) issue_s(j + 2);
             }
         }
     } else {
@@ -311,7 +313,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             m_run = m_use;
             if (j >= 1 && __any_sync(0xffffffffu, grow)) {
                 // O is rescaled only once PV_{j-1} has retired.  The signal of S_j covers
-                // PV_{j-3} (issued before it), so o_done of PV_{j-1}'s buffer is at most
+                // PV_{j-2} (issued before it), so o_done of PV_{j-1}'s buffer is at most
                 // one use behind and its parity identifies the phase.
                 mbar_wait(smem_u32(&bars->o_done[(j - 1) % kSBuf]), ((j - 1) / kSBuf) & 1, abort, a.status, 7);
                 tc_fence_after();
@@ -325,6 +327,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
                     tmem_st32(tmem + lane_addr + col, o);
                 }
+            }
+            if (ct == 0) {
+                // the release of P_j also vouches for the operands of the MMAs that
+                // follow it: V_j (PV_j) and K_{j+2} (S_{j+2}); each barrier's next use
+                // needs MMAs issued after this release, so the phases are unambiguous
+                mbar_wait(smem_u32(&bars->v_full[j % NV]), (j / NV) & 1, abort, a.status, 5);
+                if (j + 2 < nk)
+                    mbar_wait(smem_u32(&bars->k_full[(j + 2) % NK]), ((j + 2) / NK) & 1, abort, a.status, 3);
             }
             tmem_wait_st();
             tc_fence_before();
