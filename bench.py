@@ -12,7 +12,9 @@ region.
 
 Prints one JSON line (rank 0).  `value` is unmasked attention TFLOP/s (fwd + bwd
 FLOPs over the device-timed step); `e2e` is the same metric through the public
-API with pinned host buffers, host<->device copies inside the timed region.
+API with pinned host buffers, host<->device copies inside the timed region (on two
+copy streams: dO is uploaded while the forward runs, O and lse are downloaded while
+the backward runs).
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 N > 1 runs independent replicas (every CP rank is virtual, on one GPU).
 """
@@ -305,20 +307,45 @@ def run_native(args):
         h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo_))
         d2h = sum(x.numel() * x.element_size() for x in h_out)
 
+        # Copies run on two copy streams so that they overlap the kernels: dO goes up
+        # while the forward runs, O and lse come down while the backward runs.
+        s_up = torch.cuda.Stream(dev)
+        s_down = torch.cuda.Stream(dev)
+
         def e2e_step():
-            for d_, h_ in zip((dq_in, dk_in, dv_in, ddo_in), (hq_, hk_, hv_, hdo_)):
-                d_.copy_(h_, non_blocking=True)
+            start = torch.cuda.Event()
+            start.record(stream)
+            s_up.wait_event(start)
+            with torch.cuda.stream(s_up):
+                for d_, h_ in zip((dq_in, dk_in, dv_in), (hq_, hk_, hv_)):
+                    d_.copy_(h_, non_blocking=True)
+                qkv_in = torch.cuda.Event()
+                qkv_in.record(s_up)
+                ddo_in.copy_(hdo_, non_blocking=True)
+                do_in = torch.cuda.Event()
+                do_in.record(s_up)
+            stream.wait_event(qkv_in)
             thd.thd_kv_gather(plan, dq_in, k_rm=q_rm)
             thd.thd_kv_gather(plan, dk_in, dv_in, k_rm=k_rm, v_rm=v_rm)
-            thd.thd_kv_gather(plan, ddo_in, k_rm=do_rm)
             thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm)
-            thd.thd_cp_attn_bwd(plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, dq=dq, dk=dk, dv=dv, workspace=ws)
             thd.thd_rows_to_global(plan, o_rm, out=o_g)
+            o_ready = torch.cuda.Event()
+            o_ready.record(stream)
+            s_down.wait_event(o_ready)
+            with torch.cuda.stream(s_down):
+                for h_, d_ in zip(h_out[:2], (o_g, lse_rm)):
+                    h_.copy_(d_, non_blocking=True)
+                o_out = torch.cuda.Event()
+                o_out.record(s_down)
+            stream.wait_event(do_in)
+            thd.thd_kv_gather(plan, ddo_in, k_rm=do_rm)
+            thd.thd_cp_attn_bwd(plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, dq=dq, dk=dk, dv=dv, workspace=ws)
             thd.thd_rows_to_global(plan, dq, out=dq_g)
             thd.thd_rows_to_global(plan, dk, out=dk_g)
             thd.thd_rows_to_global(plan, dv, out=dv_g)
-            for h_, d_ in zip(h_out, (o_g, lse_rm, dq_g, dk_g, dv_g)):
+            for h_, d_ in zip(h_out[2:], (dq_g, dk_g, dv_g)):
                 h_.copy_(d_, non_blocking=True)
+            stream.wait_event(o_out)   # the step ends when every result is on the host
 
         e2e_step()
         torch.cuda.synchronize(dev)

@@ -117,8 +117,12 @@ struct DkdvLayout {
     static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// S^T and dP^T completions are signalled on three staged barriers each (step it uses
+// copy it % 3): besides the compute warpgroups, the producer recycles its Q and dO
+// stages on them, so the issuer commits twice per step, and with three copies the
+// phase the producer awaits is never ambiguous.
 struct DkdvBars {
-    uint64_t kv_full, q_full[3], q_empty[3], do_full[2], do_empty[2], s_full, dp_full, p_ready, ds_ready, acc_done;
+    uint64_t kv_full, q_full[3], do_full[2], stat_free[2], s_full[3], dp_full[3], p_ready, ds_ready, acc_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -151,14 +155,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         mbar_init(smem_u32(&bars->kv_full), 1);
         for (int s = 0; s < 3; ++s) {
             mbar_init(smem_u32(&bars->q_full[s]), 1);
-            mbar_init(smem_u32(&bars->q_empty[s]), 1);
+            mbar_init(smem_u32(&bars->s_full[s]), 1);
+            mbar_init(smem_u32(&bars->dp_full[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->do_full[s]), 1 + 32);          // expect_tx + the warp's lse/Delta stores
-            mbar_init(smem_u32(&bars->do_empty[s]), 1 + kCompute);   // c retired + Delta read by every thread
+            mbar_init(smem_u32(&bars->do_full[s]), 1 + 32);        // expect_tx + the warp's lse/Delta stores
+            mbar_init(smem_u32(&bars->stat_free[s]), kCompute);    // Delta of the stage read by every thread
         }
-        mbar_init(smem_u32(&bars->s_full), 1);
-        mbar_init(smem_u32(&bars->dp_full), 1);
         mbar_init(smem_u32(&bars->p_ready), kCompute);
         mbar_init(smem_u32(&bars->ds_ready), kCompute);
         mbar_init(smem_u32(&bars->acc_done), 1);
@@ -212,13 +215,19 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
             }
             const int qs = it % 3, ds = it & 1;
-            if (it >= 3) mbar_wait(smem_u32(&bars->q_empty[qs]), ((it / 3) - 1) & 1, abort, a.status, 21);
+            // Q(it) refills the stage d(it-3) read; b(it-2) is issued after d(it-3).
+            // dO(it) refills the stage c(it-2) read; a(it-1) is issued after c(it-2).
+            // The next use of either staged barrier needs a tile not loaded yet.
+            if (it >= 3) mbar_wait(smem_u32(&bars->dp_full[(it - 2) % 3]), ((it - 2) / 3) & 1, abort, a.status, 21);
             if (lane == 0) {
                 const uint32_t f = smem_u32(&bars->q_full[qs]);
                 mbar_arrive_expect_tx(f, kTile);
                 for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + qs * kTile + c * kBox, f, c * 64, h, row0);
             }
-            if (it >= 2) mbar_wait(smem_u32(&bars->do_empty[ds]), ((it >> 1) - 1) & 1, abort, a.status, 22);
+            if (it >= 2) {
+                mbar_wait(smem_u32(&bars->s_full[(it - 1) % 3]), ((it - 1) / 3) & 1, abort, a.status, 22);
+                mbar_wait(smem_u32(&bars->stat_free[ds]), ((it >> 1) - 1) & 1, abort, a.status, 22);
+            }
             const uint32_t f = smem_u32(&bars->do_full[ds]);
             if (lane == 0) {
                 mbar_arrive_expect_tx(f, kTile);
@@ -247,7 +256,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                     mma_ss(tA, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(q + off, 16, 1024), idKK, kk > 0);
                 }
-                mma_commit(smem_u32(&bars->s_full));
+                mma_commit(smem_u32(&bars->s_full[it % 3]));
             };
             auto issue_dp = [&](int it) {  // b: dP^T = V dO^T -> B
                 const int ds = it & 1;
@@ -259,7 +268,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                     mma_ss(tB, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(d + off, 16, 1024), idKK, kk > 0);
                 }
-                mma_commit(smem_u32(&bars->dp_full));
+                mma_commit(smem_u32(&bars->dp_full[it % 3]));
             };
             mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 25);
             tc_fence_after();
@@ -274,7 +283,6 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tDV, tA + kk * 8, smem_desc_sw128(d + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
-                if (it + 2 < n_it) mma_commit(smem_u32(&bars->do_empty[ds]));
                 // a of the next step: A is rewritten only after c has read it (issue order)
                 if (it + 1 < n_it) issue_s(it + 1);
                 // d: dK += dS^T Q, once dS^T is in B
@@ -284,7 +292,6 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tDK, tB + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
-                if (it + 3 < n_it) mma_commit(smem_u32(&bars->q_empty[qs]));
                 // b of the next step: B is rewritten only after d has read it (issue order)
                 if (it + 1 < n_it) issue_dp(it + 1);
             }
@@ -325,7 +332,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 
             // ---- phase 1: P^T = exp(S^T - lse) on this thread's 64 query columns
             mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 28);  // lse/Delta staged
-            mbar_wait(smem_u32(&bars->s_full), it & 1, abort, a.status, 29);
+            mbar_wait(smem_u32(&bars->s_full[it % 3]), (it / 3) & 1, abort, a.status, 29);
             tc_fence_after();
             float p[64];
 #pragma unroll
@@ -358,7 +365,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             mbar_arrive(smem_u32(&bars->p_ready));
 
             // ---- phase 2: dS^T = P^T (dP^T - Delta)
-            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 30);
+            mbar_wait(smem_u32(&bars->dp_full[it % 3]), (it / 3) & 1, abort, a.status, 30);
             tc_fence_after();
             uint32_t dk[32];
 #pragma unroll
@@ -378,7 +385,7 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     dk[ch * 16 + t / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
                 }
             }
-            mbar_arrive(smem_u32(&bars->do_empty[ds]));  // Delta of this stage read
+            mbar_arrive(smem_u32(&bars->stat_free[ds]));  // Delta of this stage read
             named_bar_sync(1, kCompute);  // all dP^T reads of B are done before dS^T overwrites it
             tmem_st32(tB + lane_addr + hf * 32, dk);
             tmem_wait_st();
@@ -427,8 +434,11 @@ struct DqLayout {
     static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// The producer recycles K and V stages on the (double-buffered) S signal: S_{j-1} is
+// issued after dQ_{j-3} (last reader of K_j's stage) and dP_{j-2} (last reader of
+// V_j's), so the issuer commits twice per step.
 struct DqBars {
-    uint64_t qdo_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], dp_full, dp_free, ds_ready, dq_done;
+    uint64_t qdo_full, k_full[3], v_full[2], s_full[2], dp_full, dp_free, ds_ready, dq_done;
     uint32_t tmem_base;
     int abort;
 };
@@ -455,13 +465,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->qdo_full), 1);
-        for (int s = 0; s < 3; ++s) {
-            mbar_init(smem_u32(&bars->k_full[s]), 1);
-            mbar_init(smem_u32(&bars->k_empty[s]), 1);
-        }
+        for (int s = 0; s < 3; ++s) mbar_init(smem_u32(&bars->k_full[s]), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->v_empty[s]), 1);
             mbar_init(smem_u32(&bars->s_full[s]), 1);
         }
         mbar_init(smem_u32(&bars->dp_full), 1);
@@ -502,11 +508,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int k0 = k0_next;
                 if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
                 const int ks = j % 3, vs = j & 1;
-                if (j >= 3) mbar_wait(smem_u32(&bars->k_empty[ks]), ((j / 3) - 1) & 1, abort, a.status, 41);
+                // S_{j-1} retired: dQ_{j-3} and dP_{j-2} are done.  The next use of that S
+                // barrier needs K_{j+1}, not loaded yet.
+                if (j >= 2) mbar_wait(smem_u32(&bars->s_full[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort, a.status, 41);
                 const uint32_t kf = smem_u32(&bars->k_full[ks]);
                 mbar_arrive_expect_tx(kf, kTile);
                 for (int c = 0; c < 2; ++c) tma_load_3d(&tmK, sK + ks * kTile + c * kBox, kf, c * 64, g, k0);
-                if (j >= 2) mbar_wait(smem_u32(&bars->v_empty[vs]), ((j >> 1) - 1) & 1, abort, a.status, 42);
                 const uint32_t vf = smem_u32(&bars->v_full[vs]);
                 mbar_arrive_expect_tx(vf, kTile);
                 for (int c = 0; c < 2; ++c) tma_load_3d(&tmV, sV + vs * kTile + c * kBox, vf, c * 64, g, k0);
@@ -543,7 +550,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                smem_desc_sw128(sV + vs * kTile + off, 16, 1024), idKK, kk > 0);
                     }
                     mma_commit(smem_u32(&bars->dp_full));
-                    if (j + 2 < nk) mma_commit(smem_u32(&bars->v_empty[vs]));
                 }
                 if (j >= 1) {
                     // dQ += dS_{j-1} K_{j-1}, dS from TMEM
@@ -554,7 +560,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ts(tDQ, tS + b * 128 + kk * 8, smem_desc_sw128(sK + ks * kTile + kk * 2048, kBox, 1024),
                                idTM, (jj > 0 || kk > 0));
-                    if (jj + 3 < nk) mma_commit(smem_u32(&bars->k_empty[ks]));
                 }
             }
             mma_commit(smem_u32(&bars->dq_done));
