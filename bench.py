@@ -12,9 +12,10 @@ region.
 
 Prints one JSON line (rank 0).  `value` is unmasked attention TFLOP/s (fwd + bwd
 FLOPs over the device-timed step); `e2e` is the same metric through the public
-API with pinned host buffers, host<->device copies inside the timed region (on two
-copy streams: dO is uploaded while the forward runs, O and lse are downloaded while
-the backward runs).
+API with pinned host buffers, host<->device copies inside the timed region, on two
+copy streams that overlap the kernels (each step's dO goes up during its forward,
+the next step's Q/K/V during its backward; O and lse come down during the backward,
+the gradients during the next step's forward).
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 N > 1 runs independent replicas (every CP rank is virtual, on one GPU).
 """
@@ -45,7 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -300,68 +301,96 @@ def run_native(args):
     if args.e2e_steps > 0:
         pin = dict(pin_memory=True)
         hq_, hk_, hv_, hdo_ = (x.cpu().pin_memory() for x in (q, k, v, do))
-        dq_in, dk_in, dv_in, ddo_in = (torch.empty_like(x) for x in (q, k, v, do))
+        h_in = (hq_, hk_, hv_, hdo_)
+        # Device copies of the inputs (global order) and of the gradients, two sets each:
+        # step i uses set i % 2, so step i+1's inputs go up and step i's gradients come
+        # down while the kernels of the neighbouring step run.  O and lse come down while
+        # the backward of their own step runs.  Every step copies its own inputs to the
+        # device and its results to the host; the first upload and the last download are
+        # inside the timed region.
+        in_sets = [tuple(torch.empty_like(x) for x in (q, k, v, do)) for _ in range(2)]
+        g_sets = [tuple(torch.empty_like(x) for x in (dq, dk, dv)) for _ in range(2)]
         o_g = torch.empty_like(o_rm)
-        dq_g, dk_g, dv_g = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
-        h_out = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (o_g, lse_rm, dq_g, dk_g, dv_g)]
-        h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo_))
+        h_out = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (o_g, lse_rm, dq, dk, dv)]
+        h2d = sum(x.numel() * x.element_size() for x in h_in)
         d2h = sum(x.numel() * x.element_size() for x in h_out)
-
-        # Copies run on two copy streams so that they overlap the kernels: dO goes up
-        # while the forward runs, O and lse come down while the backward runs.
         s_up = torch.cuda.Stream(dev)
         s_down = torch.cuda.Stream(dev)
 
-        def e2e_step():
-            start = torch.cuda.Event()
-            start.record(stream)
-            s_up.wait_event(start)
-            with torch.cuda.stream(s_up):
-                for d_, h_ in zip((dq_in, dk_in, dv_in), (hq_, hk_, hv_)):
-                    d_.copy_(h_, non_blocking=True)
-                qkv_in = torch.cuda.Event()
-                qkv_in.record(s_up)
-                ddo_in.copy_(hdo_, non_blocking=True)
-                do_in = torch.cuda.Event()
-                do_in.record(s_up)
-            stream.wait_event(qkv_in)
-            thd.thd_kv_gather(plan, dq_in, k_rm=q_rm)
-            thd.thd_kv_gather(plan, dk_in, dv_in, k_rm=k_rm, v_rm=v_rm)
-            thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm)
-            thd.thd_rows_to_global(plan, o_rm, out=o_g)
-            o_ready = torch.cuda.Event()
-            o_ready.record(stream)
-            s_down.wait_event(o_ready)
-            with torch.cuda.stream(s_down):
-                for h_, d_ in zip(h_out[:2], (o_g, lse_rm)):
-                    h_.copy_(d_, non_blocking=True)
-                o_out = torch.cuda.Event()
-                o_out.record(s_down)
-            stream.wait_event(do_in)
-            thd.thd_kv_gather(plan, ddo_in, k_rm=do_rm)
-            thd.thd_cp_attn_bwd(plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, dq=dq, dk=dk, dv=dv, workspace=ws)
-            thd.thd_rows_to_global(plan, dq, out=dq_g)
-            thd.thd_rows_to_global(plan, dk, out=dk_g)
-            thd.thd_rows_to_global(plan, dv, out=dv_g)
-            for h_, d_ in zip(h_out[2:], (dq_g, dk_g, dv_g)):
-                h_.copy_(d_, non_blocking=True)
-            stream.wait_event(o_out)   # the step ends when every result is on the host
+        def e2e_run(n_steps):
+            ev = lambda: torch.cuda.Event()  # noqa: E731
+            qkv_ready, do_ready, in_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+            g_ready, g_out = [ev(), ev()], [ev(), ev()]
+            o_out = None
 
-        e2e_step()
+            def upload(i):
+                st = i % 2
+                if i >= 2:
+                    s_up.wait_event(in_free[st])          # gathers of step i-2 read this set
+                with torch.cuda.stream(s_up):
+                    for d_, h_ in zip(in_sets[st][:3], h_in[:3]):
+                        d_.copy_(h_, non_blocking=True)
+                    qkv_ready[st].record(s_up)
+                    in_sets[st][3].copy_(h_in[3], non_blocking=True)
+                    do_ready[st].record(s_up)
+
+            begin = ev()
+            begin.record(stream)
+            s_up.wait_event(begin)
+            s_down.wait_event(begin)
+            upload(0)
+            for i in range(n_steps):
+                st = i % 2
+                dq_in, dk_in, dv_in, ddo_in = in_sets[st]
+                stream.wait_event(qkv_ready[st])
+                thd.thd_kv_gather(plan, dq_in, k_rm=q_rm)
+                thd.thd_kv_gather(plan, dk_in, dv_in, k_rm=k_rm, v_rm=v_rm)
+                if o_out is not None:
+                    stream.wait_event(o_out)              # O and lse of step i-1 are on the host
+                thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm)
+                thd.thd_rows_to_global(plan, o_rm, out=o_g)
+                o_ready = ev()
+                o_ready.record(stream)
+                s_down.wait_event(o_ready)
+                with torch.cuda.stream(s_down):
+                    for h_, d_ in zip(h_out[:2], (o_g, lse_rm)):
+                        h_.copy_(d_, non_blocking=True)
+                    o_out = ev()
+                    o_out.record(s_down)
+                stream.wait_event(do_ready[st])
+                thd.thd_kv_gather(plan, ddo_in, k_rm=do_rm)
+                in_free[st].record(stream)
+                if i + 1 < n_steps:
+                    upload(i + 1)
+                thd.thd_cp_attn_bwd(plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm, dq=dq, dk=dk, dv=dv, workspace=ws)
+                if i >= 2:
+                    stream.wait_event(g_out[st])          # gradients of step i-2 are on the host
+                for s_, d_ in zip((dq, dk, dv), g_sets[st]):
+                    thd.thd_rows_to_global(plan, s_, out=d_)
+                g_ready[st].record(stream)
+                s_down.wait_event(g_ready[st])
+                with torch.cuda.stream(s_down):
+                    for h_, d_ in zip(h_out[2:], g_sets[st]):
+                        h_.copy_(d_, non_blocking=True)
+                    g_out[st].record(s_down)
+            done = ev()
+            done.record(s_down)
+            stream.wait_event(done)                        # every result of every step is on the host
+
+        e2e_run(1)
         torch.cuda.synchronize(dev)
         replicas.barrier(info)
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        e2e_run(args.e2e_steps)
         a1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = replicas.max_over_ranks(info, a0.elapsed_time(a1), device=dev) / args.e2e_steps
         e2e = {"value": replicas.whole_job_rate(step_fl, info.world, e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms,
                "steps": args.e2e_steps}
-        del hq_, hk_, hv_, hdo_, h_out
+        del hq_, hk_, hv_, hdo_, h_in, h_out, in_sets, g_sets
 
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1)
     cpu = None
