@@ -132,6 +132,25 @@ def thd_cp_attn_fwd(plan: Plan, q_rm: torch.Tensor, k_rm: torch.Tensor, v_rm: to
     return out, lse
 
 
+def thd_cp_attn_fwd_mla(plan: Plan, q_rm: torch.Tensor, k_nope_rm: torch.Tensor, k_rope_rm: torch.Tensor,
+                        v_rm: torch.Tensor, *, scale: float | None = None, out: torch.Tensor | None = None,
+                        lse: torch.Tensor | None = None, stream=None):
+    """thd_cp_attn_fwd with multi-head latent attention keys in compact form: k_nope_rm
+    [T, hkv, d_nope] per head and k_rope_rm [T, d_rope] shared by every head; q_rm is
+    [T, hq, d_nope + d_rope].  Returns (o_rm, lse_rm [hq, T])."""
+    T, hq, dq = q_rm.shape
+    hkv, d_nope = k_nope_rm.shape[1], k_nope_rm.shape[2]
+    d_rope, dv = k_rope_rm.shape[-1], v_rm.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    out = torch.empty((T, hq, dv), dtype=q_rm.dtype, device=q_rm.device) if out is None else out
+    lse = torch.empty((hq, T), dtype=torch.float32, device=q_rm.device) if lse is None else lse
+    check("thd_cp_attn_fwd_mla", lib().thd_cp_attn_fwd_mla(
+        plan.handle, _ptr(q_rm), _ptr(k_nope_rm), _ptr(k_rope_rm), _ptr(v_rm), _ptr(out), _ptr(lse), hq, hkv,
+        d_nope, d_rope, dv, float(scale), _DTYPES[q_rm.dtype], _stream(stream)))
+    return out, lse
+
+
 def thd_cp_attn_bwd_workspace(plan: Plan, *, hq: int, hkv: int, dqk: int, dv: int,
                               dtype: torch.dtype = torch.bfloat16) -> int:
     n = ctypes.c_size_t()

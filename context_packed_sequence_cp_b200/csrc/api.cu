@@ -193,6 +193,41 @@ int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst, int64_
     return THD_OK;
 }
 
+int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope_rm, const void* k_rope_rm,
+                        const void* v_rm, void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, int32_t d_nope,
+                        int32_t d_rope, int32_t dv, float scale, int32_t dtype, void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!q_rm || !k_nope_rm || !k_rope_rm || !v_rm || !o_rm || !lse_rm || !std::isfinite(scale) || !(scale > 0.f))
+        return THD_ERR_INVALID_ARG;
+    if ((rc = check_heads(hq, hkv))) return rc;
+    if (dtype != THD_DTYPE_BF16 || d_nope != 128 || d_rope != 64 || dv != 128) return THD_ERR_UNSUPPORTED;
+    if (!aligned16(q_rm) || !aligned16(k_nope_rm) || !aligned16(k_rope_rm) || !aligned16(v_rm) || !aligned16(o_rm) ||
+        !aligned16(lse_rm))
+        return THD_ERR_MISALIGNED;
+    const int64_t items = plan->n_qtiles() * (int64_t)hq;
+    if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
+    CUtensorMap mq, mkn, mkr, mv;
+    if (!make_map_bf16(&mq, q_rm, plan->T, hq, d_nope + d_rope) || !make_map_bf16(&mkn, k_nope_rm, plan->T, hkv, d_nope) ||
+        !make_map_bf16(&mkr, k_rope_rm, plan->T, 1, d_rope) || !make_map_bf16(&mv, v_rm, plan->T, hkv, dv))
+        return THD_ERR_CUDA;
+    thd::FwdArgs a;
+    a.qtiles = plan->d_qtiles;
+    a.entries = plan->d_entries;
+    a.lpt = plan->d_lpt;
+    a.o = static_cast<__nv_bfloat16*>(o_rm);
+    a.lse = lse_rm;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.T = plan->T;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.status = plan->d_status;
+    if (items == 0) return THD_OK;
+    return thd::launch_fwd_mla_sm100(mq, mkn, mkr, mv, a, (int)items, static_cast<cudaStream_t>(stream))
+               ? THD_ERR_CUDA
+               : THD_OK;
+}
+
 int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm, void* o_rm,
                     float* lse_rm, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale, int32_t dtype,
                     void* stream) {

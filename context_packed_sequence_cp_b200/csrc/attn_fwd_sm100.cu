@@ -89,10 +89,14 @@ __device__ __forceinline__ int visible_prefix(int qpos, int nvalid, int kpos0, i
     return min(nvalid, kbrk + (qpos - b0 + 1));
 }
 
-template <int DQK, int DV>
+// SHARED_ROPE (DQK = 192 only): keys come in the compact form of multi-head latent
+// attention, a per-head 128-wide part (tmK) and one 64-wide rope key per token shared
+// by every head (tmKr); the third 64-column box of each key tile is read from tmKr.
+template <int DQK, int DV, bool SHARED_ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKr, FwdArgs a) {
+    static_assert(!SHARED_ROPE || DQK == 192, "the shared rope key is the third 64-column box");
     using L = FwdLayout<DQK, DV>;
     constexpr int NK = L::NK, NV = L::NV;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -144,6 +148,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             if (is_k) {
                 tma_prefetch_desc(&tmQ);
                 tma_prefetch_desc(&tmK);
+                if (SHARED_ROPE) tma_prefetch_desc(&tmKr);
                 const uint32_t qf = smem_u32(&bars->q_full);
                 mbar_arrive_expect_tx(qf, L::kQBytes);
                 for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
@@ -165,8 +170,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                         mbar_wait(smem_u32(&bars->s_full[(j - NK) % kSBuf]), ((j - NK) / kSBuf) & 1, abort, a.status, 1);
                     const uint32_t kf = smem_u32(&bars->k_full[st]);
                     mbar_arrive_expect_tx(kf, L::kKBytes);
-                    for (int c = 0; c < DQK / 64; ++c)
-                        tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
+                    for (int c = 0; c < DQK / 64; ++c) {
+                        if (SHARED_ROPE && c == 2)
+                            tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, k0);
+                        else
+                            tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
+                    }
                 } else {
                     if (j >= NV)
                         mbar_wait(smem_u32(&bars->o_done[(j - NV) % kSBuf]), ((j - NV) / kSBuf) & 1, abort, a.status, 9);
@@ -374,18 +383,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int DQK, int DV>
-int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const FwdArgs& a, int n_items,
-           cudaStream_t stream) {
+template <int DQK, int DV, bool SHARED_ROPE>
+int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr, const FwdArgs& a,
+           int n_items, cudaStream_t stream) {
     using L = FwdLayout<DQK, DV>;
     static bool configured = false;  // attribute is per device function; idempotent
     if (!configured) {
-        if (cudaFuncSetAttribute(fwd_kernel<DQK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(fwd_kernel<DQK, DV, SHARED_ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::kDynSmem) != cudaSuccess)
             return -1;
         configured = true;
     }
-    fwd_kernel<DQK, DV><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, a);
+    fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -393,9 +402,14 @@ int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, con
 
 int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const FwdArgs& a, int n_items, cudaStream_t stream) {
-    if (dqk == 128 && dv == 128) return launch<128, 128>(q, k, v, a, n_items, stream);
-    if (dqk == 192 && dv == 128) return launch<192, 128>(q, k, v, a, n_items, stream);
+    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, a, n_items, stream);
+    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, a, n_items, stream);
     return -2;
+}
+
+int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
+                         const CUtensorMap& v, const FwdArgs& a, int n_items, cudaStream_t stream) {
+    return launch<192, 128, true>(q, k_nope, v, k_rope, a, n_items, stream);
 }
 
 }  // namespace thd

@@ -27,6 +27,10 @@ struct FwdArgs {
 };
 int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const FwdArgs& a, int n_items, cudaStream_t stream);
+// Multi-head latent attention with a shared rope key: Q [T, hq, 192], K_nope [T, hkv, 128],
+// K_rope [T, 1, 64] (one per token, every head), V [T, hkv, 128].
+int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
+                         const CUtensorMap& v, const FwdArgs& a, int n_items, cudaStream_t stream);
 
 // ---- forward, fp32 SIMT --------------------------------------------------------
 struct FwdF32Args {

@@ -183,6 +183,26 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
                     int32_t dv, float scale, int32_t dtype, void* stream);
 
 /*
+ * thd_cp_attn_fwd_mla -- thd_cp_attn_fwd for multi-head latent attention whose keys
+ * are given in compact form: a per-head part and one rotary-position ("rope") key
+ * per token shared by every head.  [WHAT] lists MLA among the head layouts the path
+ * serves, in its expanded form (every head's key materialised at full width); the
+ * compact form computes the same attention with the expanded key
+ *   k[j,g,:] = concat(k_nope_rm[j,g,:], k_rope_rm[j,:])
+ * so that
+ *   S_ij = scale * (q_rm[i,h,:d_nope] . k_nope_rm[j,g,:] + q_rm[i,h,d_nope:] . k_rope_rm[j,:])
+ * with the same mask, outputs and error codes as thd_cp_attn_fwd.  The gather then
+ * moves d_nope * hkv + d_rope key elements per token instead of (d_nope + d_rope) * hkv.
+ *   q_rm [T, hq, d_nope + d_rope], k_nope_rm [T, hkv, d_nope], k_rope_rm [T, d_rope],
+ *   v_rm [T, hkv, dv], o_rm [T, hq, dv], lse_rm fp32 [hq, T].
+ *   Supported: THD_DTYPE_BF16 with (d_nope, d_rope, dv) = (128, 64, 128).
+ */
+int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope_rm,
+                        const void* k_rope_rm, const void* v_rm, void* o_rm, float* lse_rm,
+                        int32_t hq, int32_t hkv, int32_t d_nope, int32_t d_rope, int32_t dv,
+                        float scale, int32_t dtype, void* stream);
+
+/*
  * thd_cp_attn_bwd_workspace -- device workspace bytes thd_cp_attn_bwd needs for
  * these sizes (fp32 row statistics and the fp32 dQ accumulator).
  */

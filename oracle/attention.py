@@ -22,6 +22,10 @@ summed over the query heads that share a key/value head.
 
 Inputs are global THD-ordered arrays [T, heads, dim]; they are upcast exactly to
 float64.  Query rows are processed in blocks only to bound memory.
+
+MLA keys may also be given in compact form (a per-head part and one rope key per
+token shared by every head); attention_fwd_mla expands them and applies the same
+definition.
 """
 from __future__ import annotations
 
@@ -99,6 +103,24 @@ def attention_bwd(q, k, v, o, lse, do, cu_seqlens, scale: float):
 # Sampled forms: the same definition evaluated only where asked, so that outputs
 # of the full-size workloads can be checked one row at a time.
 # ----------------------------------------------------------------------------
+
+def expand_mla_keys(k_nope, k_rope):
+    """Expanded key of multi-head latent attention from its compact form: every
+    key/value head g of token t gets k[t, g] = concat(k_nope[t, g], k_rope[t]), the
+    rope key being one per token and shared by every head.  (The page serves MLA in
+    expanded form; this is the reading of what the compact form stands for.)"""
+    k_nope = _f64(k_nope)
+    k_rope = _f64(k_rope)
+    T, hkv, _ = k_nope.shape
+    rope = np.broadcast_to(k_rope.reshape(T, 1, -1), (T, hkv, k_rope.shape[-1]))
+    return np.concatenate([k_nope, rope], axis=2)
+
+
+def attention_fwd_mla(q, k_nope, k_rope, v, cu_seqlens, scale: float):
+    """Forward attention with MLA keys in compact form: the definition is the expanded
+    one, so this is attention_fwd on expand_mla_keys(k_nope, k_rope)."""
+    return attention_fwd(q, expand_mla_keys(k_nope, k_rope), v, cu_seqlens, scale)
+
 
 def _row_forward(qrow, kdoc, vdoc, scale):
     """One query row against its visible keys: (o, lse, p)."""

@@ -48,6 +48,20 @@ def test_bwd_small_layouts_full(hq, hkv, cp):
     assert_bf16_close(dv, wv, "dV")
 
 
+@pytest.mark.parametrize("lens,cp", [([2] * 64, 1), ([16] * 40, 8), ([2], 1), ([32, 16, 32], 8)])
+def test_bwd_degenerate_layouts(lens, cp):
+    """Documents of the minimum length 2*cp only, and a single two-token sequence."""
+    cu = syn.cu_seqlens_of(lens)
+    T = int(cu[-1])
+    q, k, v, do = syn.make_tensors(T, 4, 2, 128, 128, torch.bfloat16, seed=len(lens) + cp, with_do=True)
+    (dq, dk, dv), _ = run_fwd_bwd(cu, cp, q, k, v, do)
+    o, lse = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
+    wq, wk, wv = A.attention_bwd(q, k, v, o, lse, do, cu, 1 / math.sqrt(128))
+    assert_bf16_close(dq, wq, "dQ")
+    assert_bf16_close(dk, wk, "dK")
+    assert_bf16_close(dv, wv, "dV")
+
+
 def test_bwd_long_context_workload_sampled():
     """T=131072, cp=16, GQA 64/8: dQ at sampled rows, dK/dV at sampled keys (keys near
     the end of their document, where the oracle's cost per key is small), and two

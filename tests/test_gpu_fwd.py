@@ -97,6 +97,18 @@ def test_fwd_bf16_each_document_is_standalone_attention():
         assert np.abs(lse[:, s:e] - ld).max() <= LSE_MAX
 
 
+@pytest.mark.parametrize("lens,cp", [([2] * 64, 1), ([16] * 40, 8), ([2], 1), ([32, 16, 32], 8)])
+def test_fwd_bf16_degenerate_layouts(lens, cp):
+    """Documents of the minimum length 2*cp only (one-row chunks, q-tiles of a few rows),
+    and a single two-token sequence."""
+    cu = syn.cu_seqlens_of(lens)
+    q, k, v = syn.make_tensors(int(cu[-1]), 4, 2, 128, 128, torch.bfloat16, seed=len(lens) + cp)
+    o, lse, _, _ = run_forward(cu, cp, q, k, v)
+    want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
+    assert_bf16_close(o, want_o, "O")
+    assert np.abs(lse - want_l).max() <= LSE_MAX
+
+
 def test_fwd_rejects_unsupported_dims():
     import context_packed_sequence_cp_b200 as thd
     plan = thd.Plan([0, 16], 2).upload()

@@ -236,6 +236,35 @@ def test_fwd_cp_formulation_is_cp_independent(cp):
     np.testing.assert_allclose(l_g, lse, atol=1e-12, rtol=0)
 
 
+def test_mla_compact_keys_split_the_score_into_two_dot_products():
+    """Compact MLA keys: every score is the per-head dot product plus the dot product
+    with the token's shared rope key, checked pair by pair with explicit loops."""
+    cu = np.array([0, 6, 16])
+    T, hq, hkv, dn, dr, dv = 16, 4, 2, 5, 3, 4
+    g = np.random.default_rng(4)
+    q = g.standard_normal((T, hq, dn + dr))
+    kn = g.standard_normal((T, hkv, dn))
+    kr = g.standard_normal((T, dr))
+    v = g.standard_normal((T, hkv, dv))
+    scale = 0.37
+    o, lse = A.attention_fwd_mla(q, kn, kr, v, cu, scale)
+    for d in range(2):
+        s0, s1 = cu[d], cu[d + 1]
+        for h in range(hq):
+            gh = h // (hq // hkv)
+            for i in range(s0, s1):
+                sc = []
+                for j in range(s0, i + 1):
+                    a = sum(q[i, h, t] * kn[j, gh, t] for t in range(dn))
+                    b = sum(q[i, h, dn + t] * kr[j, t] for t in range(dr))
+                    sc.append(scale * (a + b))
+                sc = np.array(sc)
+                w = np.exp(sc - sc.max())
+                assert abs(lse[h, i] - (sc.max() + np.log(w.sum()))) < 1e-12
+                want = (w[:, None] * v[s0:i + 1, gh, :]).sum(0) / w.sum()
+                assert np.allclose(o[i, h], want, atol=1e-12)
+
+
 def test_gqa_with_equal_heads_is_mha():
     cu = np.array([0, 48, 128])
     q, k, v, _ = _rand(128, 4, 4, 16, 16, 4)
