@@ -246,15 +246,18 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
             constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);   // A TMEM, B MN-major
+            // descriptors: constant high word, low words advanced by a constant per K-step
+            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
+            const uint32_t klo = smem_desc_lo(sK, 16), vlo = smem_desc_lo(sV, 16);
             auto issue_s = [&](int it) {  // a: S^T = K Q^T -> A
                 const int qs = it % 3;
                 mbar_wait(smem_u32(&bars->q_full[qs]), (it / 3) & 1, abort, a.status, 23);
                 tc_fence_after();
-                const uint32_t q = sQ + qs * kTile;
+                const uint32_t qlo = smem_desc_lo(sQ + qs * kTile, 16);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tA, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(q + off, 16, 1024), idKK, kk > 0);
+                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(tA, smem_desc_of(klo + off, dhi), smem_desc_of(qlo + off, dhi), idKK, kk > 0);
                 }
                 mma_commit(smem_u32(&bars->s_full[it % 3]));
             };
@@ -262,11 +265,11 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const int ds = it & 1;
                 mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 24);
                 tc_fence_after();
-                const uint32_t d = sDO + ds * kTile;
+                const uint32_t dlo = smem_desc_lo(sDO + ds * kTile, 16);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    mma_ss(tB, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(d + off, 16, 1024), idKK, kk > 0);
+                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(tB, smem_desc_of(vlo + off, dhi), smem_desc_of(dlo + off, dhi), idKK, kk > 0);
                 }
                 mma_commit(smem_u32(&bars->dp_full[it % 3]));
             };
@@ -279,19 +282,19 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 // c: dV += P^T dO, once P^T is in A
                 mbar_wait(smem_u32(&bars->p_ready), it & 1, abort, a.status, 26);
                 tc_fence_after();
-                const uint32_t d = sDO + ds * kTile;
+                const uint32_t dlo = smem_desc_lo(sDO + ds * kTile, kBox);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDV, tA + kk * 8, smem_desc_sw128(d + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                    mma_ts(tDV, tA + kk * 8, smem_desc_of(dlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
                 // a of the next step: A is rewritten only after c has read it (issue order)
                 if (it + 1 < n_it) issue_s(it + 1);
                 // d: dK += dS^T Q, once dS^T is in B
                 mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 27);
                 tc_fence_after();
-                const uint32_t q = sQ + qs * kTile;
+                const uint32_t qlo = smem_desc_lo(sQ + qs * kTile, kBox);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDK, tB + kk * 8, smem_desc_sw128(q + kk * 2048, kBox, 1024), idTM, (it > 0 || kk > 0));
+                    mma_ts(tDK, tB + kk * 8, smem_desc_of(qlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
                 // b of the next step: B is rewritten only after d has read it (issue order)
                 if (it + 1 < n_it) issue_dp(it + 1);
             }
@@ -524,6 +527,9 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);
+            // descriptors: constant high word, low words advanced by a constant per K-step
+            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
+            const uint32_t qlo = smem_desc_lo(sQ, 16), dolo = smem_desc_lo(sDO, 16);
             mbar_wait(smem_u32(&bars->qdo_full), 0, abort, a.status, 43);
             tc_fence_after();
             for (int j = 0; j <= nk; ++j) {
@@ -532,22 +538,22 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     // S_j = Q K_j^T into S buffer b (it held dS_{j-2}, consumed by dQ_{j-2} issued earlier)
                     mbar_wait(smem_u32(&bars->k_full[ks]), (j / 3) & 1, abort, a.status, 44);
                     tc_fence_after();
+                    const uint32_t klo = smem_desc_lo(sK + ks * kTile, 16);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                        mma_ss(tS + b * 128, smem_desc_sw128(sQ + off, 16, 1024),
-                               smem_desc_sw128(sK + ks * kTile + off, 16, 1024), idKK, kk > 0);
+                        const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                        mma_ss(tS + b * 128, smem_desc_of(qlo + off, dhi), smem_desc_of(klo + off, dhi), idKK, kk > 0);
                     }
                     mma_commit(smem_u32(&bars->s_full[b]));
                     // dP_j = dO V_j^T, once dP_{j-1} has been read
                     mbar_wait(smem_u32(&bars->v_full[vs]), (j >> 1) & 1, abort, a.status, 45);
                     if (j >= 1) mbar_wait(smem_u32(&bars->dp_free), (j - 1) & 1, abort, a.status, 46);
                     tc_fence_after();
+                    const uint32_t vlo = smem_desc_lo(sV + vs * kTile, 16);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                        mma_ss(tDP, smem_desc_sw128(sDO + off, 16, 1024),
-                               smem_desc_sw128(sV + vs * kTile + off, 16, 1024), idKK, kk > 0);
+                        const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                        mma_ss(tDP, smem_desc_of(dolo + off, dhi), smem_desc_of(vlo + off, dhi), idKK, kk > 0);
                     }
                     mma_commit(smem_u32(&bars->dp_full));
                 }
@@ -556,10 +562,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int jj = j - 1, ks = jj % 3, b = jj & 1;
                     mbar_wait(smem_u32(&bars->ds_ready), jj & 1, abort, a.status, 47);
                     tc_fence_after();
+                    const uint32_t kmlo = smem_desc_lo(sK + ks * kTile, kBox);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tDQ, tS + b * 128 + kk * 8, smem_desc_sw128(sK + ks * kTile + kk * 2048, kBox, 1024),
-                               idTM, (jj > 0 || kk > 0));
+                        mma_ts(tDQ, tS + b * 128 + kk * 8, smem_desc_of(kmlo + kk * (2048 >> 4), dhi), idTM,
+                               (jj > 0 || kk > 0));
                 }
             }
             mma_commit(smem_u32(&bars->dq_done));

@@ -194,14 +194,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // only wait is for P_j: its release also vouches for V_j and K_{j+2}.
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
+            // descriptors: constant high words, low words advanced by a constant per K-step
+            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
+            const uint32_t qlo = smem_desc_lo(sQ, 16);
             auto issue_s = [&](int j) {
                 const int st = j % NK, b = j % kSBuf;
-                const uint32_t kb = sK + st * L::kKBytes;
+                const uint32_t klo = smem_desc_lo(sK + st * L::kKBytes, 16);
+                const uint32_t dst = tmem + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-                    mma_ss(tmem + b * 128, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                           idS, kk > 0);
+                    const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(dst, smem_desc_of(qlo + off, dhi), smem_desc_of(klo + off, dhi), idS, kk > 0);
                 }
                 mma_commit(smem_u32(&bars->s_full[b]));
             };
@@ -215,11 +218,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const int st = j % NV, b = j % kSBuf;
                 mbar_wait(smem_u32(&bars->p_full[b]), (j / kSBuf) & 1, abort, a.status, 4);
                 tc_fence_after();
-                const uint32_t vb = sV + st * L::kVBytes;
+                const uint32_t vlo = smem_desc_lo(sV + st * L::kVBytes, L::kBox);
+                const uint32_t pa = tmem + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tmem + kTmemO, tmem + b * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, L::kBox, 1024),
-                           idPV, (j > 0 || kk > 0));
+                    mma_ts(tmem + kTmemO, pa + kk * 8, smem_desc_of(vlo + kk * (2048 >> 4), dhi), idPV,
+                           (j > 0 || kk > 0));
                 mma_commit(smem_u32(&bars->o_done[b]));
                 if (j + 2 < nk) issue_s(j + 2);
             }
