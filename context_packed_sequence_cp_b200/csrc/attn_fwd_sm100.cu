@@ -8,21 +8,20 @@
 // causal attention with EOD reset.
 //
 // One CTA computes one (query tile, query head) work item, items taken in
-// longest-first order.  Warp roles (352 threads):
+// longest-first order.  Warp roles (384 threads):
 //   warp 0      TMA producer of the Q tile and of K of every listed entry;
 //   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
-//               boxes of 64 columns).
-//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of three TMEM
-//               score buffers, running two tiles ahead of O += P_j V_j (P read
-//               from TMEM).  The MMA warp observes the release of P_j several
-//               hundred cycles after the softmax signals it (measured in place);
-//               the spare third buffer keeps that latency off the softmax's path.
-//               Every barrier wait or commit between MMA groups lets the tensor
-//               pipe's short queue run dry (measured: ~60-140 cycles each), so
-//               the issuer waits once per tile (P_j released) and commits twice
-//               (PV_j retired, S_{j+2} written); the producers recycle their
-//               stages on those same two signals, and one softmax thread checks
-//               that V_j and K_{j+2} have landed before it releases P_j.
+//               boxes of 64 columns); a stage is refilled once the MMA that read
+//               it retired (K on the S signal, V on the PV signal).
+//   warp 1      TMEM owner and issuer of S_j = Q K_j^T into one of three TMEM
+//               score buffers, up to three tiles ahead of the softmax;
+//   warp 11     issuer of O += P_j V_j (P read from TMEM).
+//               The tensor pipe's queue is short: with one issuing thread every
+//               barrier wait or commit between MMA groups let it run dry, and the
+//               issuing thread competed for its SMSP with two softmax warps
+//               (measured in place: ~95-140 cycles per 128x128x16 MMA against 64).
+//               Two issuers on different SMSPs keep it fed (measured 64 cycles per
+//               MMA under the same load).
 //   warps 3-10  two softmax warpgroups; a thread owns half of one query row: it
 //               reads its 64 columns of S_j from TMEM, masks PARTIAL entries only,
 //               keeps the running max / sum in fp32 (base-2, scale folded in; the
@@ -43,7 +42,8 @@ constexpr int BM = 128, BN = 128, kMaxStages = 3;
 constexpr int kSBuf = 3;                 // S/P buffers in TMEM
 constexpr uint32_t kTmemO = kSBuf * 128; // first O column
 constexpr int kSoftmax = 256;          // two softmax warpgroups
-constexpr int kThreads = 96 + kSoftmax;  // K producer, MMA issuer, V producer, softmax
+constexpr int kPvWarp = 3 + kSoftmax / 32;  // PV issuer, after the softmax warps
+constexpr int kThreads = 96 + kSoftmax + 32; // K producer, S issuer, V producer, softmax, PV issuer
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -186,49 +186,54 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kPvWarp) {
+        // ---------------------------------------------------- MMA issuers
+        // Two issuing threads on different SMSPs keep the tensor pipe's short queue fed
+        // while either of them waits or commits: warp 1 issues every S_j, warp kPvWarp
+        // every PV_j.  Each waits only for what its own MMAs need:
+        //   S_j:  K_j landed, and PV_{j-3} retired (S_j's TMEM buffer held P_{j-3}).
+        //         The next use of that o_done barrier is PV_j, which needs S_j: the
+        //         awaited phase is unambiguous.
+        //   PV_j: P_j released (which implies S_j retired) and V_j landed.
         if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            // Order: S_0, S_1, then per tile PV_j followed by S_{j+2}.  S_{j+2} reuses the
-            // TMEM buffer of P_{j-1} after PV_{j-1} (issue order).  Inside the loop the
-            // only wait is for P_j: its release also vouches for V_j and K_{j+2}.
-            constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
-            constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
-            // descriptors: constant high words, low words advanced by a constant per K-step
             constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
-            const uint32_t qlo = smem_desc_lo(sQ, 16);
-            auto issue_s = [&](int j) {
-                const int st = j % NK, b = j % kSBuf;
-                const uint32_t klo = smem_desc_lo(sK + st * L::kKBytes, 16);
-                const uint32_t dst = tmem + b * 128;
+            if (warp == 1) {
+                constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+                const uint32_t qlo = smem_desc_lo(sQ, 16);
+                mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
+                for (int j = 0; j < nk; ++j) {
+                    const int st = j % NK, b = j % kSBuf;
+                    if (j >= kSBuf)
+                        mbar_wait(smem_u32(&bars->o_done[b]), ((j - kSBuf) / kSBuf) & 1, abort, a.status, 10);
+                    mbar_wait(smem_u32(&bars->k_full[st]), (j / NK) & 1, abort, a.status, 3);
+                    tc_fence_after();
+                    const uint32_t klo = smem_desc_lo(sK + st * L::kKBytes, 16);
+                    const uint32_t dst = tmem + b * 128;
 #pragma unroll
-                for (int kk = 0; kk < DQK / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
-                    mma_ss(dst, smem_desc_of(qlo + off, dhi), smem_desc_of(klo + off, dhi), idS, kk > 0);
+                    for (int kk = 0; kk < DQK / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
+                        mma_ss(dst, smem_desc_of(qlo + off, dhi), smem_desc_of(klo + off, dhi), idS, kk > 0);
+                    }
+                    mma_commit(smem_u32(&bars->s_full[b]));
                 }
-                mma_commit(smem_u32(&bars->s_full[b]));
-            };
-            mbar_wait(smem_u32(&bars->q_full), 0, abort, a.status, 2);
-            for (int j = 0; j < 2 && j < nk; ++j) {
-                mbar_wait(smem_u32(&bars->k_full[j % NK]), (j / NK) & 1, abort, a.status, 3);
-                tc_fence_after();
-                issue_s(j);
-            }
-            for (int j = 0; j < nk; ++j) {
-                const int st = j % NV, b = j % kSBuf;
-                mbar_wait(smem_u32(&bars->p_full[b]), (j / kSBuf) & 1, abort, a.status, 4);
-                tc_fence_after();
-                const uint32_t vlo = smem_desc_lo(sV + st * L::kVBytes, L::kBox);
-                const uint32_t pa = tmem + b * 128;
+            } else {
+                constexpr uint32_t idPV = idesc_bf16_f32(BM, DV, false, true);
+                for (int j = 0; j < nk; ++j) {
+                    const int st = j % NV, b = j % kSBuf;
+                    mbar_wait(smem_u32(&bars->p_full[b]), (j / kSBuf) & 1, abort, a.status, 4);
+                    mbar_wait(smem_u32(&bars->v_full[st]), (j / NV) & 1, abort, a.status, 5);
+                    tc_fence_after();
+                    const uint32_t vlo = smem_desc_lo(sV + st * L::kVBytes, L::kBox);
+                    const uint32_t pa = tmem + b * 128;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tmem + kTmemO, pa + kk * 8, smem_desc_of(vlo + kk * (2048 >> 4), dhi), idPV,
-                           (j > 0 || kk > 0));
-                mma_commit(smem_u32(&bars->o_done[b]));
-                if (j + 2 < nk) issue_s(j + 2);
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_ts(tmem + kTmemO, pa + kk * 8, smem_desc_of(vlo + kk * (2048 >> 4), dhi), idPV,
+                               (j > 0 || kk > 0));
+                    mma_commit(smem_u32(&bars->o_done[b]));
+                }
             }
         }
-    } else {
+    } else if (warp >= 3 && warp < 3 + kSoftmax / 32) {
         // ---------------------------------------------------- softmax warpgroups
         // Two warpgroups; thread (row, half) owns 64 of the row's 128 score columns
         // and DV/2 of its output columns.  Row maxima are combined through shared
@@ -340,14 +345,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
                     tmem_st32(tmem + lane_addr + col, o);
                 }
-            }
-            if (ct == 0) {
-                // the release of P_j also vouches for the operands of the MMAs that
-                // follow it: V_j (PV_j) and K_{j+2} (S_{j+2}); each barrier's next use
-                // needs MMAs issued after this release, so the phases are unambiguous
-                mbar_wait(smem_u32(&bars->v_full[j % NV]), (j / NV) & 1, abort, a.status, 5);
-                if (j + 2 < nk)
-                    mbar_wait(smem_u32(&bars->k_full[(j + 2) % NK]), ((j + 2) / NK) & 1, abort, a.status, 3);
             }
             tmem_wait_st();
             tc_fence_before();
