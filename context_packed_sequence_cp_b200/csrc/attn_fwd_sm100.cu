@@ -76,6 +76,10 @@ struct Bars {
 // Number of leading key columns of an entry visible to a query at global position
 // qpos: key t sits at kpos0 + t + (t >= kbrk ? kjump : 0), positions increase with
 // t, so the visible keys are a prefix of the nvalid listed ones.
+// Pair barriers: the two threads that hold the halves of a row sit in warps w and w+4
+// (the same TMEM lane quarter), so every exchange between halves, and every overwrite
+// of a half's TMEM columns read by its partner, needs only those two warps: barrier
+// 2 + (w & 3), 64 threads.
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -237,7 +241,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // ---------------------------------------------------- softmax warpgroups
         // Two warpgroups; thread (row, half) owns 64 of the row's 128 score columns
         // and DV/2 of its output columns.  Row maxima are combined through shared
-        // memory once per tile (double-buffered); row sums once at the end.
+        // memory once per tile (double-buffered); row sums once at the end; the two
+        // halves of a row meet on their pair barrier only.
         const int ct = threadIdx.x - 96;
         const int hf = ct >> 7;
         const int wq = warp & 3;
@@ -303,7 +308,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const float pmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                      fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             xch[(xb * 2 + hf) * 128 + row] = pmax;
-            named_bar_sync(1, kSoftmax);  // both halves' scores are read and their maxima posted
+            named_bar_sync(2 + wq, 64);  // both halves' scores are read and their maxima posted
             const float mx = fmaxf(pmax, xch[(xb * 2 + (hf ^ 1)) * 128 + row]) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + kRescaleThreshold;
@@ -354,9 +359,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (nk > 0)
             mbar_wait(smem_u32(&bars->o_done[(nk - 1) % kSBuf]), ((nk - 1) / kSBuf) & 1, abort, a.status, 8);
         tc_fence_after();
-        named_bar_sync(1, kSoftmax);  // last maxima read before the buffer is reused for the sums
+        named_bar_sync(2 + wq, 64);  // last maxima read before the buffer is reused for the sums
         xch[hf * 128 + row] = l_run;
-        named_bar_sync(1, kSoftmax);
+        named_bar_sync(2 + wq, 64);
         const float l_tot = l_run + xch[(hf ^ 1) * 128 + row];
         const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
         __nv_bfloat16* orow = a.o + ((size_t)(row0 + row) * a.hq + h) * DV + hf * (DV / 2);
