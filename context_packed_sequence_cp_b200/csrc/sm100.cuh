@@ -173,17 +173,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, 1024-byte aligned atoms.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// The same descriptor split into its two 32-bit words, for issue loops: the high word
-// (stride byte offset, version, swizzle) is constant per operand layout, and the start
-// address field of the low word advances by (offset >> 4) per K-step.  Shared-memory
-// addresses are below 256 KB, so (addr >> 4) fits the 14-bit field and adding a step
-// offset never carries into the leading-byte-offset field.
+// Shared-memory matrix descriptor (128-byte swizzle, 1024-byte aligned atoms), built
+// as two 32-bit words for issue loops: the low word holds the start address >> 4
+// (bits 0-13) and the leading byte offset >> 4 (bits 16-29); the high word the stride
+// byte offset >> 4 (bits 32-45), version 1 (bit 46) and swizzle mode 2 (bits 61-63).
+// The high word is constant per operand layout, and the start field of the low word
+// advances by (offset >> 4) per K-step.  Shared-memory addresses are below 256 KB, so
+// (addr >> 4) fits the 14-bit field and a step offset never carries into the
+// leading-byte-offset field.
 __device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
     return ((saddr >> 4) & 0x3FFF) | (((lbo_bytes >> 4) & 0x3FFF) << 16);
 }
