@@ -86,6 +86,29 @@ class Plan:
             pass
 
 
+def thd_cu_seqlens_from_eod(tokens, eod_id: int) -> np.ndarray:
+    """Document boundaries of an EOD-delimited packed sequence (host int32 token ids):
+    a document ends with, and includes, each EOD token; the tokens after the last EOD
+    form a final document.  Returns cu_seqlens as an int32 array."""
+    tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).ravel())
+    n = ctypes.c_int32(0)
+    rc = lib().thd_cu_seqlens_from_eod(_i32p(tok), tok.size, int(eod_id), None, 0, ctypes.byref(n))
+    if rc not in (0, -9):
+        check("thd_cu_seqlens_from_eod", rc)
+    cu = np.zeros(n.value + 1, dtype=np.int32)
+    check("thd_cu_seqlens_from_eod", lib().thd_cu_seqlens_from_eod(
+        _i32p(tok), tok.size, int(eod_id), _i32p(cu), cu.size, ctypes.byref(n)))
+    return cu
+
+
+def thd_position_ids(cu_seqlens) -> np.ndarray:
+    """Per-document position ids: token t of document d gets t - cu_seqlens[d]."""
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    pos = np.zeros(int(cu[-1]) if cu.size else 0, dtype=np.int32)
+    check("thd_position_ids", lib().thd_position_ids(_i32p(cu), cu.size - 1, _i32p(pos)))
+    return pos
+
+
 def thd_cp_plan(cu_seqlens, cp: int) -> Plan:
     return Plan(cu_seqlens, cp)
 

@@ -364,7 +364,9 @@ const char* thd_cp_strerror(int code) {
         case THD_ERR_CUDA: return "CUDA runtime or launch error";
         case THD_ERR_UNSUPPORTED: return "unsupported dtype / head dimension combination";
         case THD_ERR_ALLOC: return "allocation failed";
-        case THD_ERR_TOO_LARGE: return "hq * T exceeds the fixed scratch of the no-allocation backward";
+        case THD_ERR_TOO_LARGE:
+            return "result does not fit: hq * T exceeds the fixed scratch of the no-allocation backward, "
+                   "or the caller's output array is too small";
         default: return "unknown error";
     }
 }

@@ -50,7 +50,8 @@ extern "C" {
 #define THD_ERR_CUDA          -6  /* a CUDA runtime call or a launch failed         */
 #define THD_ERR_UNSUPPORTED   -7  /* dtype / head-dim combination not built         */
 #define THD_ERR_ALLOC         -8  /* host or device allocation failed               */
-#define THD_ERR_TOO_LARGE     -9  /* hq * T exceeds the fixed scratch of thd_cp_attn_bwd_noalloc */
+#define THD_ERR_TOO_LARGE     -9  /* result does not fit: hq * T beyond the fixed scratch of
+                                      thd_cp_attn_bwd_noalloc, or a caller's array too small */
 
 /* ---- element types ----------------------------------------------------- */
 #define THD_DTYPE_BF16 0   /* bf16 inputs, fp32 accumulation, tcgen05 tensor cores */
@@ -75,6 +76,32 @@ typedef struct thd_cp_plan_info_s {
     int64_t n_entries;  /* listed (query tile, key tile) pairs                   */
     int64_t causal_pairs; /* sum over documents of L (L + 1) / 2                 */
 } thd_cp_plan_info_t;
+
+/*
+ * thd_cu_seqlens_from_eod -- document boundaries of an EOD-delimited packed
+ * sequence ([USER] EOD attention-mask reset): a document ends with, and includes,
+ * each token equal to eod_id; the tokens after the last EOD form a final document.
+ *   tokens      host int32[T], T >= 1 (and T <= INT32_MAX).
+ *   cu_seqlens  host int32[capacity]: receives n_docs + 1 offsets, cu_seqlens[0] = 0,
+ *               cu_seqlens[n_docs] = T, strictly increasing.
+ *   n_docs      receives the number of documents, also when capacity is too small,
+ *               so that a caller may size the array with a first call.
+ * Errors: THD_ERR_INVALID_ARG (null tokens/n_docs, T out of range, capacity < 0),
+ * THD_ERR_TOO_LARGE (cu_seqlens null or capacity < n_docs + 1; *n_docs set).
+ * Host only; the divisibility rule of thd_cp_plan is not checked here.
+ */
+int thd_cu_seqlens_from_eod(const int32_t* tokens, int64_t T, int32_t eod_id, int32_t* cu_seqlens,
+                            int32_t capacity, int32_t* n_docs);
+
+/*
+ * thd_position_ids -- per-document position ids of the packed tokens ([USER]: the
+ * position of a token restarts with its document): pos[t] = t - cu_seqlens[d] for
+ * cu_seqlens[d] <= t < cu_seqlens[d+1].
+ *   cu_seqlens  host int32[n_docs + 1], n_docs >= 1; pos host int32[cu_seqlens[n_docs]].
+ * Errors: THD_ERR_INVALID_ARG, THD_ERR_BAD_SEQLENS (cu_seqlens[0] != 0 or not strictly
+ * increasing).  Host only.
+ */
+int thd_position_ids(const int32_t* cu_seqlens, int32_t n_docs, int32_t* pos);
 
 /*
  * thd_cp_plan -- validate a packed layout and build the symmetric partition and
