@@ -392,6 +392,24 @@ def run_native(args):
                "steps": args.e2e_steps}
         del hq_, hk_, hv_, hdo_, h_in, h_out, in_sets, g_sets
 
+    # ------------------------------------------------ rotary embedding (SURVEY-next row; outside the step)
+    # Per-document positions of the workload's layout, applied in place to a copy of Q:
+    # 2 * T * hq * dqk * 2 bytes of HBM traffic per call (read + write) plus the table.
+    pos_d = torch.from_numpy(thd.thd_position_ids(cu)).to(dev)
+    q_rope = q.clone()
+    rope_ws = torch.empty(T * (w.dqk // 2) * 8, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        thd.thd_rope_apply(q_rope, pos_d, workspace=rope_ws)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(5):
+        thd.thd_rope_apply(q_rope, pos_d, workspace=rope_ws)
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    rope_ms = r0.elapsed_time(r1) / 5
+    rope_bytes = 2 * T * w.hq * w.dqk * 2 + T * (w.dqk // 2) * 8 * 2 + 4 * T
+    del q_rope, rope_ws
+
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1)
     cpu = None
     if info.rank == 0 and info.world == 1 and not args.no_cpu_baseline:
@@ -424,6 +442,9 @@ def run_native(args):
                      "flops_per_launch": bwd_fl},
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac_of_peak": fwd_tf / sustained, "flops": fwd_fl},
         "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac_of_peak": bwd_tf / sustained, "flops": bwd_fl},
+        "rope": {"ms": rope_ms, "gbs": rope_bytes / (rope_ms / 1e3) / 1e9,
+                 "frac_of_hbm": rope_bytes / (rope_ms / 1e3) / 1e9 / hbm, "bytes": rope_bytes,
+                 "note": "thd_rope_apply on Q with per-document positions, outside the timed step"},
         "gather": {"ms": gather_ms, "gbs": gather_gbs, "frac_of_hbm": gather_gbs / hbm, "bytes": gather_bytes,
                    "hbm_peak_gbs": hbm, "peak_source": peak_src},
         "e2e": e2e,

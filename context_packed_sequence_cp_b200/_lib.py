@@ -36,6 +36,9 @@ SIGNATURES = {
     "thd_cp_attn_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _F, _I32, _P]),
     "thd_cu_seqlens_from_eod": (ctypes.c_int, [_P, ctypes.c_int64, _I32, _P, _I32, _P]),
     "thd_position_ids": (ctypes.c_int, [_P, _I32, _P]),
+    "thd_rope_workspace": (ctypes.c_int, [ctypes.c_int64, _I32, _P]),
+    "thd_rope_apply": (ctypes.c_int, [_P, _P, ctypes.c_int64, _I32, _I32, _I32, ctypes.c_double, _I32, _P,
+                                      ctypes.c_size_t, _P]),
     "thd_cp_attn_fwd_mla": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _F, _I32,
                                            _P]),
     "thd_cp_attn_bwd_workspace": (ctypes.c_int, [_P, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(ctypes.c_size_t)]),

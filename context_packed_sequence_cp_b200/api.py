@@ -109,6 +109,22 @@ def thd_position_ids(cu_seqlens) -> np.ndarray:
     return pos
 
 
+def thd_rope_apply(x: torch.Tensor, pos: torch.Tensor, *, rot_dim: int | None = None, base: float = 10000.0,
+                   workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rotary position embedding (half-split) in place on bf16 x [T, heads, dim] with
+    per-row positions pos (device int32 [T]); returns x."""
+    T, heads, dim = x.shape
+    rot_dim = dim if rot_dim is None else int(rot_dim)
+    n = ctypes.c_size_t()
+    check("thd_rope_workspace", lib().thd_rope_workspace(T, rot_dim, ctypes.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(int(n.value), dtype=torch.uint8, device=x.device)
+    check("thd_rope_apply", lib().thd_rope_apply(
+        _ptr(x), _ptr(pos), T, heads, dim, rot_dim, float(base), _DTYPES[x.dtype], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return x
+
+
 def thd_cp_plan(cu_seqlens, cp: int) -> Plan:
     return Plan(cu_seqlens, cp)
 

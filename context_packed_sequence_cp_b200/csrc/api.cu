@@ -182,6 +182,28 @@ int thd_kv_gather(thd_cp_plan_t plan, const void* k, const void* v, void* k_rm, 
     return THD_OK;
 }
 
+int thd_rope_workspace(int64_t T, int32_t rot_dim, size_t* bytes) {
+    if (!bytes || T < 1 || rot_dim < 2 || (rot_dim & 1)) return THD_ERR_INVALID_ARG;
+    *bytes = (size_t)T * (size_t)(rot_dim / 2) * sizeof(float2);
+    return THD_OK;
+}
+
+int thd_rope_apply(void* x, const int32_t* pos, int64_t T, int32_t heads, int32_t dim, int32_t rot_dim,
+                   double base, int32_t dtype, void* workspace, size_t ws_bytes, void* stream) {
+    if (!x || !pos || !workspace || T < 1 || heads < 1 || dim < 2 || rot_dim < 2 || (rot_dim & 1) ||
+        rot_dim > dim || !std::isfinite(base) || !(base > 0.0))
+        return THD_ERR_INVALID_ARG;
+    if (dtype != THD_DTYPE_BF16) return THD_ERR_UNSUPPORTED;
+    size_t need = 0;
+    thd_rope_workspace(T, rot_dim, &need);
+    if (ws_bytes < need) return THD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(pos) || !aligned16(workspace)) return THD_ERR_MISALIGNED;
+    return thd::launch_rope(static_cast<__nv_bfloat16*>(x), pos, T, heads, dim, rot_dim, base,
+                            static_cast<float2*>(workspace), num_sms_current(), static_cast<cudaStream_t>(stream))
+               ? THD_ERR_CUDA
+               : THD_OK;
+}
+
 int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst, int64_t row_bytes, void* stream) {
     int rc = ready(plan);
     if (rc) return rc;

@@ -72,4 +72,8 @@ struct BwdArgs {
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream);
 
+// ---- rotary position embedding (half-split), per-document positions ---------------
+int launch_rope(__nv_bfloat16* x, const int32_t* pos, int64_t T, int heads, int dim, int rot_dim, double base,
+                float2* table, int num_sms, cudaStream_t stream);
+
 }  // namespace thd

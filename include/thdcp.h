@@ -104,6 +104,31 @@ int thd_cu_seqlens_from_eod(const int32_t* tokens, int64_t T, int32_t eod_id, in
 int thd_position_ids(const int32_t* cu_seqlens, int32_t n_docs, int32_t* pos);
 
 /*
+ * thd_rope_workspace -- bytes of the cos/sin table thd_rope_apply needs:
+ * T * (rot_dim / 2) * 8.  Errors: THD_ERR_INVALID_ARG.
+ */
+int thd_rope_workspace(int64_t T, int32_t rot_dim, size_t* bytes);
+
+/*
+ * thd_rope_apply -- rotary position embedding with per-document positions, in place
+ * ([USER]: positions restart with every EOD-delimited document; the pages name no
+ * rotary variant -- this is the half-split form).  For every row t and head h, and
+ * i < rot_dim / 2, with angle = pos[t] * base^(-2 i / rot_dim):
+ *   x[t,h,i]             <- x[t,h,i] cos - x[t,h,i + rot_dim/2] sin
+ *   x[t,h,i + rot_dim/2] <- x[t,h,i + rot_dim/2] cos + x[t,h,i] sin
+ * dimensions rot_dim .. dim-1 unchanged.  The angles are formed in double precision
+ * into a fp32 cos/sin table (the workspace), then applied to every head.
+ *   x          device bf16 [T, heads, dim] (any row order; pos gives each row's position).
+ *   pos        device int32[T] (e.g. thd_position_ids copied to the device).
+ *   rot_dim    even, 2 <= rot_dim <= dim.  base > 0.
+ *   workspace  device, >= thd_rope_workspace bytes, 16-byte aligned; caller-owned.
+ * Errors: THD_ERR_INVALID_ARG, THD_ERR_UNSUPPORTED (dtype other than bf16),
+ * THD_ERR_MISALIGNED, THD_ERR_CUDA.
+ */
+int thd_rope_apply(void* x, const int32_t* pos, int64_t T, int32_t heads, int32_t dim, int32_t rot_dim,
+                   double base, int32_t dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * thd_cp_plan -- validate a packed layout and build the symmetric partition and
  * the per-tile metadata ([USER] divisibility rule; [WHAT] EOD-aware symmetric
  * partitioning and metadata caching).

@@ -1,6 +1,7 @@
-"""Document boundaries from EOD tokens and per-document position ids: the fp64-free
-oracle (oracle/eod.py) pinned by a hand-derived example and invariants, then the
-library's host entry points compared with it bit for bit.  CPU only."""
+"""Document boundaries from EOD tokens and per-document position ids: the oracle
+(oracle/eod.py) pinned by a hand-derived example and invariants, then the library's
+host entry points compared with it bit for bit; and the rotary-embedding oracle
+(oracle/rope.py) pinned by properties that fix the rotation.  CPU only."""
 import os
 
 import numpy as np
@@ -101,3 +102,41 @@ def test_library_errors():
     with pytest.raises(thd.ThdError) as e:
         thd.thd_position_ids([0, 3, 3])                                                  # empty document
     assert e.value.kind == "BAD_SEQLENS"
+
+
+# ---------------------------------------------------------------- rotary embedding oracle
+from oracle import rope as R   # noqa: E402
+
+
+def _rand_x(T, H, D, seed):
+    return np.random.default_rng(seed).standard_normal((T, H, D))
+
+
+def test_rope_is_complex_rotation():
+    """Each pair (x_i, x_{i+R/2}) as the complex number x_i + j x_{i+R/2}, multiplied by
+    exp(j * pos * base^(-2i/R)); dimensions past R untouched."""
+    T, H, D, Rd = 7, 2, 10, 8
+    x = _rand_x(T, H, D, 1)
+    pos = np.array([0, 1, 5, 17, 300, 65535, 2])
+    y = R.rope(x, pos, Rd, 500.0)
+    for i in range(Rd // 2):
+        z = (x[:, :, i] + 1j * x[:, :, i + Rd // 2]) * np.exp(1j * pos[:, None] * 500.0 ** (-2 * i / Rd))
+        assert np.allclose(y[:, :, i], z.real, atol=1e-12) and np.allclose(y[:, :, i + Rd // 2], z.imag, atol=1e-12)
+    assert np.array_equal(y[:, :, Rd:], x[:, :, Rd:])
+
+
+def test_rope_position_zero_is_identity_and_norms_are_kept():
+    x = _rand_x(5, 3, 16, 2)
+    assert np.allclose(R.rope(x, np.zeros(5), 16), x, atol=0)
+    y = R.rope(x, np.arange(5) * 1000, 16)
+    h = 8
+    assert np.allclose(x[:, :, :h] ** 2 + x[:, :, h:] ** 2, y[:, :, :h] ** 2 + y[:, :, h:] ** 2, atol=1e-12)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    q = _rand_x(1, 1, 16, 3)
+    k = _rand_x(1, 1, 16, 4)
+    def score(m, n):
+        return float((R.rope(q, [m], 16) * R.rope(k, [n], 16)).sum())
+    for m, n, d in [(5, 2, 100), (40000, 39000, 7), (9, 9, 123)]:
+        assert abs(score(m, n) - score(m + d, n + d)) < 1e-9
