@@ -193,7 +193,7 @@ int thd_rope_apply(void* x, const int32_t* pos, int64_t T, int32_t heads, int32_
     if (!x || !pos || !workspace || T < 1 || heads < 1 || dim < 2 || rot_dim < 2 || (rot_dim & 1) ||
         rot_dim > dim || !std::isfinite(base) || !(base > 0.0))
         return THD_ERR_INVALID_ARG;
-    if (dtype != THD_DTYPE_BF16) return THD_ERR_UNSUPPORTED;
+    if (dtype != THD_DTYPE_BF16 || (rot_dim % 16) || (dim % 8)) return THD_ERR_UNSUPPORTED;
     size_t need = 0;
     thd_rope_workspace(T, rot_dim, &need);
     if (ws_bytes < need) return THD_ERR_INVALID_ARG;

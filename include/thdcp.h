@@ -120,7 +120,8 @@ int thd_rope_workspace(int64_t T, int32_t rot_dim, size_t* bytes);
  * into a fp32 cos/sin table (the workspace), then applied to every head.
  *   x          device bf16 [T, heads, dim] (any row order; pos gives each row's position).
  *   pos        device int32[T] (e.g. thd_position_ids copied to the device).
- *   rot_dim    even, 2 <= rot_dim <= dim.  base > 0.
+ *   rot_dim    even, 2 <= rot_dim <= dim, base > 0; built for rot_dim % 16 == 0 and
+ *              dim % 8 == 0 (16-byte accesses), THD_ERR_UNSUPPORTED otherwise.
  *   workspace  device, >= thd_rope_workspace bytes, 16-byte aligned; caller-owned.
  * Errors: THD_ERR_INVALID_ARG, THD_ERR_UNSUPPORTED (dtype other than bf16),
  * THD_ERR_MISALIGNED, THD_ERR_CUDA.
