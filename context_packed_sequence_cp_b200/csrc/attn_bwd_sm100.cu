@@ -659,15 +659,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
-    static bool configured = false;
-    if (!configured) {
-        if (cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvLayout::kBytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqLayout::kBytes) !=
-                cudaSuccess)
-            return -1;
-        configured = true;
-    }
+    static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};
+    if (!ensure_dynamic_smem(dkdv_kernel, DkdvLayout::kBytes, dkdv_configured) ||
+        !ensure_dynamic_smem(dq_kernel, DqLayout::kBytes, dq_configured))
+        return -1;
     bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
     dkdv_kernel<<<(unsigned)((int64_t)n_tiles * a.hkv), kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);

@@ -393,13 +393,8 @@ template <int DQK, int DV, bool SHARED_ROPE>
 int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr, const FwdArgs& a,
            int n_items, cudaStream_t stream) {
     using L = FwdLayout<DQK, DV>;
-    static bool configured = false;  // attribute is per device function; idempotent
-    if (!configured) {
-        if (cudaFuncSetAttribute(fwd_kernel<DQK, DV, SHARED_ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::kDynSmem) != cudaSuccess)
-            return -1;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};
+    if (!ensure_dynamic_smem(fwd_kernel<DQK, DV, SHARED_ROPE>, L::kDynSmem, configured)) return -1;
     fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

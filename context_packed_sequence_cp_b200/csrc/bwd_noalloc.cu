@@ -56,30 +56,6 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// [rows, heads, dim] bf16 viewed as 64-column x 1-head x 128-row boxes, 128-byte swizzle.
-bool map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return false;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    const cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
-    const cuuint64_t strides[2] = {(cuuint64_t)dim * 2, (cuuint64_t)heads * dim * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm,
@@ -101,8 +77,8 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     int rc = scratch_on_current_device(&delta);
     if (rc != THD_OK) return rc;
     CUtensorMap mq, mk, mv, mdo;
-    if (!map_bf16(&mq, q_rm, plan->T, hq, dqk) || !map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
-        !map_bf16(&mv, v_rm, plan->T, hkv, dv) || !map_bf16(&mdo, do_rm, plan->T, hq, dv))
+    if (!thd::make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !thd::make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
+        !thd::make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !thd::make_map_bf16(&mdo, do_rm, plan->T, hq, dv))
         return THD_ERR_CUDA;
     thd::BwdArgs a;
     a.qtiles = plan->d_qtiles;

@@ -1,11 +1,32 @@
 // Launch interfaces between the C ABI layer (api.cu) and the device kernels.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace thd {
+
+// True once `fn` may use `bytes` of dynamic shared memory on the current device.  The
+// attribute belongs to the device's context, so it is set once per device (devices
+// 0-63 are remembered in `done`, others are set on every call); two host threads that
+// race on the first call may both set it, which is harmless.
+template <typename Kernel>
+inline bool ensure_dynamic_smem(Kernel* fn, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    if (bit) done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
+
+// [rows, heads, dim] bf16 tensor viewed as a 3-D TMA map with 64-column x 1-head x
+// 128-row boxes and 128-byte swizzle (the layout the tcgen05 descriptors expect).
+// False when the driver's encoder is unavailable or rejects the map.
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
 
 // ---- row gather (all-gather layout, and its inverse) -----------------------
 // dst_t[j] = src_t[idx[j]] for whole rows of row_bytes_t bytes, t = 0, 1 (the second
