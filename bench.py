@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -48,6 +49,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None, help="where the nvidia-smi clock samples go (default: a temp file)")
     return ap.parse_args()
 
 
@@ -157,10 +159,10 @@ class ClockSampler:
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, bus_id: str):
+    def __init__(self, bus_id: str, path: str | None = None):
         self.bus = bus_id.lower()
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(), f"thdcp_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -273,7 +275,7 @@ def run_native(args):
     if plan.device_status() != 0:
         raise RuntimeError("a kernel's bounded wait gave up during warm-up")
 
-    sampler = ClockSampler(bus_id_of(dev))
+    sampler = ClockSampler(bus_id_of(dev), args.clocks_csv)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     replicas.barrier(info)
     torch.cuda.synchronize(dev)
@@ -392,7 +394,7 @@ def run_native(args):
                "steps": args.e2e_steps}
         del hq_, hk_, hv_, hdo_, h_in, h_out, in_sets, g_sets
 
-    # ------------------------------------------------ rotary embedding (SURVEY-next row; outside the step)
+    # ------------------------------------------------ rotary embedding (reported beside the step, not in it)
     # Per-document positions of the workload's layout, applied in place to a copy of Q:
     # 2 * T * hq * dqk * 2 bytes of HBM traffic per call (read + write) plus the table.
     pos_d = torch.from_numpy(thd.thd_position_ids(cu)).to(dev)
