@@ -34,3 +34,15 @@ def test_reference_arm_prints_the_contract_line():
 def test_reference_arm_runs_on_rank_zero_only():
     r = _run({"RANK": "1"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_plan_timing_on_the_benchmark_layout():
+    """The host plan that the bench line reports under "plan" builds the long-context layout
+    (cp=16, T=131072) on the CPU and closes every plan it timed."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import context_packed_sequence_cp_b200 as thd
+    from context_packed_sequence_cp_b200 import synthetic as syn
+    cu = syn.cu_seqlens_of(syn.doc_lengths(bench.WORKLOAD, 0))
+    ms = bench.time_plan(thd, cu, syn.WORKLOADS[bench.WORKLOAD].cp, reps=2)
+    assert 0 < ms < 10_000
