@@ -22,7 +22,6 @@
 
 #include <algorithm>
 #include <limits>
-#include <utility>
 #include <vector>
 
 namespace {
@@ -115,7 +114,20 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         const int64_t n_tiles = tile_base.back();
         if (n_tiles > std::numeric_limits<int32_t>::max()) return THD_ERR_INVALID_ARG;
         p->qtiles.assign((size_t)n_tiles * THD_QTILE_FIELDS, 0);
-        p->entries.clear();
+
+        // Entry count first, so that the entry table is sized once and filled in place.
+        int64_t n_entries = 0;
+        for (int r = 0; r < cp; ++r)
+            for (int d = 0; d < n_docs; ++d) {
+                const int64_t nseg = 2 * lay.chunk(d);
+                for (int64_t u0 = 0; u0 < nseg; u0 += BM) {
+                    const int64_t qmax = lay.pos(r, d, std::min<int64_t>(u0 + BM, nseg) - 1);
+                    for (int rk = 0; rk < cp; ++rk) n_entries += ceil_div(lay.visible_prefix(rk, d, qmax), BN);
+                }
+            }
+        if (n_entries > std::numeric_limits<int32_t>::max() / 2) return THD_ERR_INVALID_ARG;
+        p->entries.assign((size_t)n_entries * THD_ENTRY_FIELDS, 0);
+        int64_t ne_fill = 0;
 
         for (int r = 0; r < cp; ++r)
             for (int d = 0; d < n_docs; ++d) {
@@ -125,12 +137,12 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
                     const int64_t u0 = i * BM, m = std::min<int64_t>(BM, nseg - u0);
                     const int64_t qmin = lay.pos(r, d, u0), qmax = lay.pos(r, d, u0 + m - 1);
                     int32_t* q = &p->qtiles[(size_t)ti * THD_QTILE_FIELDS];
-                    const int64_t first = p->n_entries();
+                    const int64_t first = ne_fill;
                     for (int rk = 0; rk < cp; ++rk) {
                         const int64_t v = lay.visible_prefix(rk, d, qmax);
                         for (int64_t j = 0; j * BN < v; ++j) {
                             const int64_t k0u = j * BN, nv = std::min<int64_t>(BN, v - k0u);
-                            int32_t e[THD_ENTRY_FIELDS];
+                            int32_t* e = &p->entries[(size_t)ne_fill++ * THD_ENTRY_FIELDS];
                             e[0] = (int32_t)(lay.seg_row(rk, d) + k0u);
                             e[1] = (int32_t)nv;
                             int32_t enc[3];
@@ -141,7 +153,6 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
                             e[5] = lay.pos(rk, d, k0u + nv - 1) <= qmin ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
                             e[6] = (int32_t)(tile_base[(size_t)rk * n_docs + d] + j);
                             e[7] = rk;
-                            p->entries.insert(p->entries.end(), e, e + THD_ENTRY_FIELDS);
                         }
                     }
                     int32_t enc[3];
@@ -154,13 +165,12 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
                     q[5] = enc[1];
                     q[6] = enc[2];
                     q[7] = (int32_t)qmax;
-                    q[8] = (int32_t)(p->n_entries() - first);
+                    q[8] = (int32_t)(ne_fill - first);
                     q[9] = (int32_t)first;
                     q[10] = (int32_t)s[d];
                     q[11] = (int32_t)(s[d] + L[d]);
                 }
             }
-        if (p->n_entries() > std::numeric_limits<int32_t>::max() / 2) return THD_ERR_INVALID_ARG;
 
         // ---- longest-first order of query tiles ------------------------------
         p->lpt.resize(n_tiles);
@@ -170,41 +180,33 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         });
 
         // ---- key-tile transpose for the backward (counting sort by key tile) --
-        const int64_t ne = p->n_entries();
+        // Each key tile's list is in descending order of the query tile's last
+        // position, ties (which cannot occur within one document) by tile index.  A
+        // key tile sees exactly the query tiles of its document whose last position is
+        // at or past its first key, so every list is a prefix of one per-document
+        // order, and key tiles walked at the same time read the same query tiles.
+        // Walking the query tiles once in that order makes the counting-sort fill
+        // emit every list already sorted.
+        const int64_t ne = n_entries;
         p->kt_off.assign(n_tiles + 1, 0);
         for (int64_t e = 0; e < ne; ++e) p->kt_off[p->entries[(size_t)e * THD_ENTRY_FIELDS + 6] + 1]++;
         for (int64_t t = 0; t < n_tiles; ++t) p->kt_off[t + 1] += p->kt_off[t];
+        std::vector<int32_t> by_last(n_tiles);
+        for (int64_t t = 0; t < n_tiles; ++t) by_last[t] = (int32_t)t;
+        std::sort(by_last.begin(), by_last.end(), [&](int32_t a, int32_t b) {
+            const int32_t pa = p->qtiles[(size_t)a * THD_QTILE_FIELDS + 7];
+            const int32_t pb = p->qtiles[(size_t)b * THD_QTILE_FIELDS + 7];
+            return pa != pb ? pa > pb : a < b;
+        });
         std::vector<int32_t> fill(p->kt_off.begin(), p->kt_off.end() - 1);
         p->kt_list.assign((size_t)ne * 2, 0);
-        for (int64_t qt = 0; qt < n_tiles; ++qt) {
+        for (const int32_t qt : by_last) {
             const int32_t* q = &p->qtiles[(size_t)qt * THD_QTILE_FIELDS];
             for (int64_t e = q[9]; e < (int64_t)q[9] + q[8]; ++e) {
                 const int32_t kt = p->entries[(size_t)e * THD_ENTRY_FIELDS + 6];
                 const int32_t at = fill[kt]++;
-                p->kt_list[(size_t)at * 2] = (int32_t)qt;
+                p->kt_list[(size_t)at * 2] = qt;
                 p->kt_list[(size_t)at * 2 + 1] = (int32_t)e;
-            }
-        }
-        // Each list in descending order of the query tile's last position (ties,
-        // which cannot occur within one document, by tile index).  A key tile sees
-        // exactly the query tiles of its document whose last position is at or past
-        // its first key, so every key tile's list is a prefix of one per-document
-        // order: key tiles walked at the same time read the same query tiles.
-        for (int64_t kt = 0; kt < n_tiles; ++kt) {
-            std::vector<std::pair<int32_t, int32_t>> run;
-            for (int64_t at = p->kt_off[kt]; at < p->kt_off[kt + 1]; ++at)
-                run.emplace_back(p->kt_list[(size_t)at * 2], p->kt_list[(size_t)at * 2 + 1]);
-            std::sort(run.begin(), run.end(), [&](const std::pair<int32_t, int32_t>& x,
-                                                  const std::pair<int32_t, int32_t>& y) {
-                const int32_t px = p->qtiles[(size_t)x.first * THD_QTILE_FIELDS + 7];
-                const int32_t py = p->qtiles[(size_t)y.first * THD_QTILE_FIELDS + 7];
-                return px != py ? px > py : x.first < y.first;
-            });
-            int64_t at = p->kt_off[kt];
-            for (const auto& pr : run) {
-                p->kt_list[(size_t)at * 2] = pr.first;
-                p->kt_list[(size_t)at * 2 + 1] = pr.second;
-                ++at;
             }
         }
         p->kt_lpt.resize(n_tiles);
