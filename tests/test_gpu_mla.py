@@ -71,7 +71,7 @@ def test_mla_compact_keys_equal_expanded_keys_exactly():
 
 def test_mla_rejects_other_widths():
     plan = thd.Plan([0, 16], 2).upload()
-    q = torch.zeros(16, 2, 192, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(16, 2, 160, dtype=torch.bfloat16, device="cuda")
     kn = torch.zeros(16, 2, 128, dtype=torch.bfloat16, device="cuda")
     kr = torch.zeros(16, 32, dtype=torch.bfloat16, device="cuda")   # rope width 32: not built
     with pytest.raises(thd.ThdError) as e:
