@@ -181,8 +181,10 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
  * thd_cp_plan_upload -- copy the tables to the current device once and keep them
  * there ([WHAT] metadata caching).  Allocates device memory owned by the plan
  * (freed by thd_cp_plan_destroy) and enqueues the copies on `stream`; the host
- * tables stay valid.  Calling it again is a no-op.  Errors: THD_ERR_CUDA,
- * THD_ERR_ALLOC.
+ * tables stay valid.  Calling it again is a no-op.  The tables live on the device
+ * that is current here; every later call with this plan launches on the current
+ * device and must be made with that same device current, on buffers of that device.
+ * Errors: THD_ERR_CUDA, THD_ERR_ALLOC.
  */
 int thd_cp_plan_upload(thd_cp_plan_t plan, void* stream);
 
