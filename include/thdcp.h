@@ -287,7 +287,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
 
 /*
  * thd_cp_attn_bwd_noalloc -- thd_cp_attn_bwd for callers that cannot allocate
- * device memory.  (The paper has no counterpart: this is a deployment variant of
+ * device memory.  (The source page has no counterpart: this is a deployment variant of
  * the same backward.)  thd_cp_attn_bwd wants a workspace for the per-row
  * statistic Delta; a caller whose device memory is owned entirely by another
  * allocator, or whose hot path may not call cudaMalloc (it can synchronise the
