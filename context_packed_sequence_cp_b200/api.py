@@ -127,9 +127,13 @@ class Plan:
         return out
 
     def upload(self, stream=None) -> "Plan":
+        """Copies the tables to the current device; a second call is a no-op, as in the
+        library, and the tables stay on the device of the first."""
+        first = not self.uploaded
         check("thd_cp_plan_upload", lib().thd_cp_plan_upload(self._h, _stream(stream)))
-        self.uploaded = True
-        self.device = _current_device()
+        if first:
+            self.uploaded = True
+            self.device = _current_device()
         return self
 
     def device_status(self, reset: bool = True) -> int:

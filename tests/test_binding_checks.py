@@ -200,3 +200,13 @@ def test_not_uploaded_comes_first(rec):
     with pytest.raises(_lib.ThdError) as e:
         thd.thd_cp_attn_fwd(plan, None, None, None)
     assert _kind(e) == "NOT_UPLOADED" and rec.calls == []
+
+
+def test_second_upload_keeps_the_first_device(rec, monkeypatch):
+    cu = [0, 64]
+    plan = thd.Plan(cu, 2)
+    plan.upload()
+    assert plan.uploaded and plan.device == 0 and rec.calls == ["thd_cp_plan_upload"]
+    monkeypatch.setattr(api, "_current_device", lambda: 1)
+    plan.upload()
+    assert plan.device == 0
