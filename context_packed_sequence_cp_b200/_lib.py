@@ -30,6 +30,7 @@ SIGNATURES = {
     "thd_cp_plan_info": (ctypes.c_int, [_P, _P]),
     "thd_cp_plan_export": (ctypes.c_int, [_P, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32]),
     "thd_cp_plan_upload": (ctypes.c_int, [_P, _P]),
+    "thd_cp_plan_update": (ctypes.c_int, [_P, _PI32, _I32, _I32, _P]),
     "thd_cp_plan_destroy": (None, [_P]),
     "thd_kv_gather": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _P]),
     "thd_rows_to_global": (ctypes.c_int, [_P, _P, _P, _I64, _P]),

@@ -102,12 +102,7 @@ class Plan:
         h = ctypes.c_void_p()
         check("thd_cp_plan", lib().thd_cp_plan(_i32p(cu), int(cu.size - 1), int(cp), ctypes.byref(h)))
         self._h = h
-        self.cu_seqlens = cu
-        info = PlanInfo()
-        check("thd_cp_plan_info", lib().thd_cp_plan_info(self._h, ctypes.byref(info)))
-        self.T, self.cp, self.n_docs = int(info.T), int(info.cp), int(info.n_docs)
-        self.Tl, self.n_qtiles, self.n_entries = int(info.Tl), int(info.n_qtiles), int(info.n_entries)
-        self.causal_pairs = int(info.causal_pairs)
+        self._refresh(cu)
         self.uploaded = False
         self.device = None
 
@@ -135,6 +130,37 @@ class Plan:
             self.uploaded = True
             self.device = _current_device()
         return self
+
+    def update(self, cu_seqlens, cp: int | None = None, stream=None) -> "Plan":
+        """thd_cp_plan_update: re-plan in place for a new layout (a new batch).  The host
+        tables are rebuilt; if the plan was uploaded, the new tables are copied to its
+        device on `stream` (the current stream by default), in stream order, without a
+        device-wide synchronisation."""
+        fn = "thd_cp_plan_update"
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        cp = self.cp if cp is None else int(cp)
+        if self.uploaded:
+            dev = _current_device()
+            if dev != self.device:
+                _bad(fn, f"the plan's tables are on cuda:{self.device}, the current device is cuda:{dev}")
+            s = _stream(stream)
+        else:
+            s = ctypes.c_void_p(0)
+        rc = lib().thd_cp_plan_update(self._h, _i32p(cu), int(cu.size - 1), cp, s)
+        if rc != 0 and rc in (_CODE["CUDA"], _CODE["ALLOC"]):
+            self.uploaded = False
+        if rc == 0 or rc in (_CODE["CUDA"], _CODE["ALLOC"]):
+            self._refresh(cu)
+        check(fn, rc)
+        return self
+
+    def _refresh(self, cu):
+        self.cu_seqlens = cu
+        info = PlanInfo()
+        check("thd_cp_plan_info", lib().thd_cp_plan_info(self._h, ctypes.byref(info)))
+        self.T, self.cp, self.n_docs = int(info.T), int(info.cp), int(info.n_docs)
+        self.Tl, self.n_qtiles, self.n_entries = int(info.Tl), int(info.n_qtiles), int(info.n_entries)
+        self.causal_pairs = int(info.causal_pairs)
 
     def device_status(self, reset: bool = True) -> int:
         v = ctypes.c_int32()

@@ -2,6 +2,7 @@
 // lifecycle with cached device tables, TMA descriptor encoding and kernel launches.
 // No entry point falls back to another implementation: an unsupported shape is an
 // error, and every computation runs in this library's kernels.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -28,23 +29,100 @@ int check_heads(int32_t hq, int32_t hkv) {
     return THD_OK;
 }
 
+// The plan's tables must be on the device, and that device must be current: the
+// kernels launch on the current device and read the tables in place.  An error left
+// pending by earlier, unrelated work is reported here (and not cleared), so that the
+// launch checks after this point see only this library's launches.
 int ready(thd_plan* p) {
     if (!p) return THD_ERR_INVALID_ARG;
     if (!p->uploaded) return THD_ERR_NOT_UPLOADED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+    if (dev != p->device) return THD_ERR_INVALID_ARG;
+    if (cudaPeekAtLastError() != cudaSuccess) return THD_ERR_CUDA;
     return THD_OK;
 }
 
+// Frees the device and pinned host memory of a plan.  The caller has made the plan's
+// device current and waited for every kernel that reads the tables.
 void free_device(thd_plan* p) {
-    int32_t** ptrs[] = {&p->d_q_idx, &p->d_rm_of_global, &p->d_qtiles, &p->d_entries,
-                        &p->d_lpt,   &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt, &p->d_status};
-    for (auto pp : ptrs) {
-        if (*pp) cudaFree(*pp);
-        *pp = nullptr;
+    if (p->d_buf) cudaFree(p->d_buf);
+    p->d_buf = nullptr;
+    p->d_cap = 0;
+    for (int i = 0; i < 2; ++i) {
+        if (p->staged[i]) cudaEventDestroy(p->staged[i]);
+        if (p->h_stage[i]) cudaFreeHost(p->h_stage[i]);
+        p->staged[i] = nullptr;
+        p->h_stage[i] = nullptr;
+        p->h_cap[i] = 0;
     }
+    p->d_q_idx = p->d_rm_of_global = p->d_qtiles = p->d_entries = p->d_lpt = nullptr;
+    p->d_kt_off = p->d_kt_list = p->d_kt_lpt = p->d_status = nullptr;
     p->uploaded = false;
 }
 
+constexpr size_t kAlign = 256;
+size_t round_up(size_t n) { return (n + kAlign - 1) & ~(kAlign - 1); }
+
+// Copies every host table into the plan's device allocation on `s`: through one of
+// the two pinned staging buffers (waiting only for the copy that last used it) and
+// one cudaMemcpyAsync.  The device allocation grows, in stream order, when the
+// tables outgrow it; the status word at its start survives a re-plan.  Work on `s`
+// enqueued earlier reads the previous tables before the copy overwrites them.
+int copy_tables(thd_plan* p, cudaStream_t s, bool first) {
+    const std::vector<int32_t>* src[] = {&p->q_idx,  &p->rm_of_global, &p->qtiles,  &p->entries,
+                                         &p->lpt,    &p->kt_off,       &p->kt_list, &p->kt_lpt};
+    int32_t** dst[] = {&p->d_q_idx, &p->d_rm_of_global, &p->d_qtiles,  &p->d_entries,
+                       &p->d_lpt,   &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt};
+    size_t off[8];
+    size_t total = kAlign;  // the status word (16 bytes) sits in the first 256
+    for (int i = 0; i < 8; ++i) {
+        off[i] = total;
+        total += round_up(std::max<size_t>(src[i]->size(), 4) * sizeof(int32_t));
+    }
+    const int st = p->next_stage;
+    if (!p->staged[st] && cudaEventCreateWithFlags(&p->staged[st], cudaEventDisableTiming) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (cudaEventSynchronize(p->staged[st]) != cudaSuccess) return THD_ERR_CUDA;
+    if (p->h_cap[st] < total) {
+        if (p->h_stage[st]) cudaFreeHost(p->h_stage[st]);
+        p->h_stage[st] = nullptr;
+        p->h_cap[st] = 0;
+        const size_t cap = total + total / 4;
+        if (cudaHostAlloc(&p->h_stage[st], cap, cudaHostAllocDefault) != cudaSuccess) return THD_ERR_ALLOC;
+        p->h_cap[st] = cap;
+    }
+    uint8_t* h = static_cast<uint8_t*>(p->h_stage[st]);
+    for (int i = 0; i < 8; ++i)
+        if (!src[i]->empty()) std::memcpy(h + off[i], src[i]->data(), src[i]->size() * sizeof(int32_t));
+    if (p->d_cap < total) {
+        void* fresh = nullptr;
+        const size_t cap = total + total / 4;
+        if (cudaMallocAsync(&fresh, cap, s) != cudaSuccess) return THD_ERR_ALLOC;
+        if (p->d_buf) {
+            // the status word moves with the tables; the old buffer is released after
+            // every earlier reader on this stream
+            if (cudaMemcpyAsync(fresh, p->d_buf, 16, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+                cudaFreeAsync(p->d_buf, s) != cudaSuccess)
+                return THD_ERR_CUDA;
+        }
+        p->d_buf = fresh;
+        p->d_cap = cap;
+    }
+    uint8_t* d = static_cast<uint8_t*>(p->d_buf);
+    if (first && cudaMemsetAsync(d, 0, 16, s) != cudaSuccess) return THD_ERR_CUDA;
+    if (cudaMemcpyAsync(d + kAlign, h + kAlign, total - kAlign, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return THD_ERR_CUDA;
+    if (cudaEventRecord(p->staged[st], s) != cudaSuccess) return THD_ERR_CUDA;
+    p->next_stage = st ^ 1;
+    p->d_status = reinterpret_cast<int32_t*>(d);
+    for (int i = 0; i < 8; ++i) *dst[i] = reinterpret_cast<int32_t*>(d + off[i]);
+    return THD_OK;
+}
+
 }  // namespace
+
+int thd_plan_ready(thd_cp_plan_s* p) { return ready(p); }
 
 namespace thd {
 
@@ -129,45 +207,67 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
 int thd_cp_plan_upload(thd_cp_plan_t plan, void* stream) {
     if (!plan) return THD_ERR_INVALID_ARG;
     if (plan->uploaded) return THD_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    struct Item {
-        int32_t** dst;
-        const std::vector<int32_t>* src;
-    } items[] = {{&plan->d_q_idx, &plan->q_idx},     {&plan->d_rm_of_global, &plan->rm_of_global},
-                 {&plan->d_qtiles, &plan->qtiles},   {&plan->d_entries, &plan->entries},
-                 {&plan->d_lpt, &plan->lpt},         {&plan->d_kt_off, &plan->kt_off},
-                 {&plan->d_kt_list, &plan->kt_list}, {&plan->d_kt_lpt, &plan->kt_lpt}};
-    for (auto& it : items) {
-        const size_t bytes = std::max<size_t>(it.src->size(), 4) * sizeof(int32_t);
-        if (cudaMalloc(it.dst, bytes) != cudaSuccess) {
-            free_device(plan);
-            return THD_ERR_ALLOC;
-        }
-        if (!it.src->empty() &&
-            cudaMemcpyAsync(*it.dst, it.src->data(), it.src->size() * sizeof(int32_t), cudaMemcpyHostToDevice,
-                            s) != cudaSuccess) {
-            free_device(plan);
-            return THD_ERR_CUDA;
-        }
-    }
-    if (cudaMalloc(&plan->d_status, 16) != cudaSuccess) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+    const int rc = copy_tables(plan, static_cast<cudaStream_t>(stream), true);
+    if (rc != THD_OK) {
+        cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
         free_device(plan);
-        return THD_ERR_ALLOC;
+        return rc;
     }
-    if (cudaMemsetAsync(plan->d_status, 0, 16, s) != cudaSuccess) {
-        free_device(plan);
-        return THD_ERR_CUDA;
-    }
-    cudaGetDevice(&plan->device);
+    plan->device = dev;
     plan->uploaded = true;
     return THD_OK;
 }
 
-void thd_cp_plan_destroy(thd_cp_plan_t plan) {
-    if (!plan) return;
+int thd_cp_plan_update(thd_cp_plan_t plan, const int32_t* cu_seqlens, int32_t n_docs, int32_t cp, void* stream) {
+    if (!plan) return THD_ERR_INVALID_ARG;
     if (plan->uploaded) {
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+        if (dev != plan->device) return THD_ERR_INVALID_ARG;
+    }
+    thd_plan fresh;
+    const int rc = thd_build_plan(cu_seqlens, n_docs, cp, &fresh);
+    if (rc != THD_OK) return rc;
+    plan->T = fresh.T;
+    plan->Tl = fresh.Tl;
+    plan->cp = fresh.cp;
+    plan->n_docs = fresh.n_docs;
+    plan->causal_pairs = fresh.causal_pairs;
+    plan->doc_start.swap(fresh.doc_start);
+    plan->doc_len.swap(fresh.doc_len);
+    plan->q_idx.swap(fresh.q_idx);
+    plan->rm_of_global.swap(fresh.rm_of_global);
+    plan->qtiles.swap(fresh.qtiles);
+    plan->entries.swap(fresh.entries);
+    plan->lpt.swap(fresh.lpt);
+    plan->kt_off.swap(fresh.kt_off);
+    plan->kt_list.swap(fresh.kt_list);
+    plan->kt_lpt.swap(fresh.kt_lpt);
+    if (!plan->uploaded) return THD_OK;
+    // On a failed copy the device tables no longer match the host tables: the plan
+    // becomes not-uploaded, and a later thd_cp_plan_upload copies them afresh.
+    const int cr = copy_tables(plan, static_cast<cudaStream_t>(stream), false);
+    if (cr != THD_OK) {
         cudaDeviceSynchronize();
         free_device(plan);
+    }
+    return cr;
+}
+
+void thd_cp_plan_destroy(thd_cp_plan_t plan) {
+    if (!plan) return;
+    if (plan->uploaded || plan->d_buf || plan->h_stage[0] || plan->h_stage[1]) {
+        // Free on the device that holds the tables, after every kernel there that may
+        // still read them; the caller's current device is restored afterwards.
+        int prev = -1;
+        const bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+        const bool switched = plan->device >= 0 && (!have_prev || prev != plan->device) &&
+                              cudaSetDevice(plan->device) == cudaSuccess;
+        cudaDeviceSynchronize();
+        free_device(plan);
+        if (switched && have_prev) cudaSetDevice(prev);
     }
     delete plan;
 }
@@ -373,10 +473,15 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
 int thd_cp_device_status(thd_cp_plan_t plan, int32_t reset, int32_t* status) {
     if (!plan || !status) return THD_ERR_INVALID_ARG;
     if (!plan->uploaded) return THD_ERR_NOT_UPLOADED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return THD_ERR_CUDA;
+    if (dev != plan->device) return THD_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return THD_ERR_CUDA;
     int32_t v = 0;
     if (cudaMemcpy(&v, plan->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return THD_ERR_CUDA;
     *status = v;
-    if (reset && cudaMemset(plan->d_status, 0, sizeof(int32_t)) != cudaSuccess) return THD_ERR_CUDA;
+    if (reset && (cudaMemset(plan->d_status, 0, sizeof(int32_t)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess))
+        return THD_ERR_CUDA;
     return THD_OK;
 }
 

@@ -62,8 +62,8 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
                                        const void* o_rm, const float* lse_rm, const void* do_rm, float* dq_rm,
                                        float* dk_rm, float* dv_rm, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv,
                                        float scale, int32_t dtype, void* stream) {
-    if (!plan) return THD_ERR_INVALID_ARG;
-    if (!plan->uploaded) return THD_ERR_NOT_UPLOADED;
+    int rc = thd_plan_ready(plan);
+    if (rc != THD_OK) return rc;
     if (!q_rm || !k_rm || !v_rm || !o_rm || !lse_rm || !do_rm || !dq_rm || !dk_rm || !dv_rm ||
         !std::isfinite(scale) || !(scale > 0.f))
         return THD_ERR_INVALID_ARG;
@@ -74,7 +74,7 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     for (const void* p : ptrs)
         if (!aligned16(p)) return THD_ERR_MISALIGNED;
     float* delta = nullptr;
-    int rc = scratch_on_current_device(&delta);
+    rc = scratch_on_current_device(&delta);
     if (rc != THD_OK) return rc;
     CUtensorMap mq, mk, mv, mdo;
     if (!thd::make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !thd::make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||

@@ -17,10 +17,14 @@
  *
  * Conventions shared by every entry point
  *   - Return value: THD_OK (0) or a negative THD_ERR_* code.  On an argument or
- *     layout error nothing is launched and no output is touched.
+ *     layout error nothing is launched and no output is touched.  A launching entry
+ *     point that finds a CUDA error already pending from earlier, unrelated work
+ *     returns THD_ERR_CUDA without launching and leaves that error pending for its
+ *     owner; THD_ERR_CUDA after a launch is this library's own.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Device entry points only enqueue work: they never synchronise and
- *     never allocate device memory, except thd_cp_plan_upload (see there).
+ *     never allocate device memory, except thd_cp_plan_upload and
+ *     thd_cp_plan_update (see there).
  *   - Device buffers are owned by the caller; the library reads and writes them
  *     only inside the enqueued kernels.  Device pointers must be 16-byte aligned
  *     (THD_ERR_MISALIGNED otherwise).
@@ -179,17 +183,43 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
 
 /*
  * thd_cp_plan_upload -- copy the tables to the current device once and keep them
- * there ([WHAT] metadata caching).  Allocates device memory owned by the plan
- * (freed by thd_cp_plan_destroy) and enqueues the copies on `stream`; the host
- * tables stay valid.  Calling it again is a no-op.  The tables live on the device
- * that is current here; every later call with this plan launches on the current
- * device and must be made with that same device current, on buffers of that device.
+ * there ([WHAT] metadata caching).  The plan owns one stream-ordered device
+ * allocation (cudaMallocAsync on `stream`) holding every table and its status word,
+ * and two pinned host staging buffers; the tables reach the device by one
+ * cudaMemcpyAsync on `stream`.  The host tables stay valid.  Calling it again is a
+ * no-op.  The tables live on the device that is current here; every later call with
+ * this plan must be made with that same device current, on buffers of that device
+ * (a launching call made with another device current returns THD_ERR_INVALID_ARG).
  * Errors: THD_ERR_CUDA, THD_ERR_ALLOC.
  */
 int thd_cp_plan_upload(thd_cp_plan_t plan, void* stream);
 
-/* Release the plan and its device tables (synchronises the device first if
- * tables were uploaded).  NULL is ignored. */
+/*
+ * thd_cp_plan_update -- re-plan in place for a new packed layout (a new batch):
+ * rebuilds the partition and the tile tables for (cu_seqlens, n_docs, cp), with the
+ * validation and errors of thd_cp_plan, and, if the plan was uploaded, copies them to
+ * its device on `stream` ([WHAT] metadata caching: the cache is refreshed, not
+ * rebuilt, when the layout changes).  No device-wide synchronisation: the copy goes
+ * through one of the plan's two pinned staging buffers (the host waits only for the
+ * copy issued two updates earlier, which normally finished long ago), into the
+ * plan's device allocation, which grows in stream order (cudaMallocAsync /
+ * cudaFreeAsync on `stream`) only when the new tables do not fit.
+ * Ordering: the copy overwrites the tables in place, after all work enqueued on
+ * `stream` before this call; work that uses the plan on other streams must be
+ * ordered before this call's position on `stream` by the caller.  Calls made after
+ * it read the new layout.  The device status word is kept.
+ * On a validation error the plan is unchanged.  If the device copy fails
+ * (THD_ERR_CUDA / THD_ERR_ALLOC), the host tables hold the new layout and the plan
+ * is left not uploaded.  With the plan uploaded, its device must be current
+ * (THD_ERR_INVALID_ARG otherwise).
+ */
+int thd_cp_plan_update(thd_cp_plan_t plan, const int32_t* cu_seqlens, int32_t n_docs,
+                       int32_t cp, void* stream);
+
+/* Release the plan and its device tables.  If tables were uploaded, the plan's device
+ * is made current, synchronised (so that no kernel still reads the tables) and the
+ * caller's current device restored.  NULL is ignored.  A training loop that re-plans
+ * every batch calls thd_cp_plan_update instead and destroys once. */
 void thd_cp_plan_destroy(thd_cp_plan_t plan);
 
 /*
@@ -302,7 +332,10 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
  *   that device current) and caches it; make that first call before any stream
  *   capture.  All calls share the array: calls whose kernels overlap on the GPU
  *   (e.g. on different streams) race on it and must be serialised by the caller.
- *   The array is fully rewritten by each call before it is read.
+ *   The array is fully rewritten by each call before it is read.  The cached
+ *   address belongs to the device's current context: after cudaDeviceReset on a
+ *   device, this entry point must not be called on that device again in the same
+ *   process (the array then has a new address the cache does not know).
  */
 #define THD_NOALLOC_MAX_ROWS_X_HEADS 8388608
 int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, const void* v_rm,

@@ -85,3 +85,33 @@ def test_device_entry_points_refuse_before_upload():
     with pytest.raises(ThdError) as e:
         thd_cp_attn_fwd(plan, x, x, x, stream=type("S", (), {"cuda_stream": 0})())
     assert e.value.kind == "NOT_UPLOADED"
+
+
+def test_plan_update_equals_a_fresh_plan():
+    """thd_cp_plan_update re-plans in place: after every update (larger, smaller, another
+    cp) the exported tables are bit-identical to a freshly built plan's and to the
+    oracle's; an invalid layout leaves the plan as it was."""
+    rng = np.random.default_rng(77)
+    plan = Plan([0, 16], 2)
+    for i in range(12):
+        cp = int(rng.choice([1, 2, 4, 8]))
+        lens = syn.random_lengths(rng, 4000 if i % 3 else 400, 2 * cp, max_docs=7)
+        cu = syn.cu_seqlens_of(lens)
+        plan.update(cu, cp)
+        fresh = Plan(cu, cp)
+        ex, ref = plan.export(), fresh.export()
+        want = TT.tile_plan(cu, cp)
+        assert (plan.T, plan.cp, plan.n_qtiles, plan.n_entries) == (fresh.T, fresh.cp, fresh.n_qtiles,
+                                                                     fresh.n_entries)
+        for k in KEYS:
+            assert np.array_equal(ex[k], ref[k]), k
+            assert np.array_equal(ex[k], want[k].reshape(ex[k].shape)), k
+        fresh.close()
+    before = plan.export()
+    with pytest.raises(ThdError) as e:
+        plan.update([0, 6, 12], 2)          # 6 is not a multiple of 2 * cp = 4
+    assert e.value.kind == "NOT_DIVISIBLE"
+    after = plan.export()
+    for k in KEYS:
+        assert np.array_equal(before[k], after[k]), k
+    plan.close()
