@@ -192,6 +192,65 @@ def attention_bwd_keys(q, k, v, do, cu_seqlens, scale, keys, kv_heads):
     return dK, dV
 
 
+def attention_bwd_key_blocks(q, k, v, do, cu_seqlens, scale, blocks, kv_heads):
+    """dK and dV of contiguous key blocks of one document, by a blocked pass over the
+    query rows that can see them.  ``blocks`` is a list of (first key, number of keys),
+    all inside one document; returns lists dK[b] [n, len(kv_heads), Dqk] and
+    dV[b] [n, len(kv_heads), Dv].
+
+    The same definition as attention_bwd, evaluated where asked: for each query head h
+    of a key/value head's group and each block of query rows i (from the first key of
+    the earliest block to the document's end), the full row of scores against keys
+    s .. i gives lse_i, P_i and O_i = P_i V, hence Delta_i = dO_i . O_i; then, for the
+    asked keys j only, dP_ij = dO_i . V_j, dS_ij = P_ij (dP_ij - Delta_i),
+    dV_j += P_ij dO_i and dK_j += scale dS_ij Q_i.  Written with float64 torch CPU
+    operations (multi-threaded), so that a 65536-token document takes seconds per
+    head rather than minutes."""
+    import torch
+
+    def t64(x):
+        return x.detach().to("cpu", torch.float64) if hasattr(x, "detach") else torch.from_numpy(_f64(x))
+
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    doc = doc_of_token(cu)
+    hq, hkv = q.shape[1], k.shape[1]
+    group = hq // hkv
+    d = int(doc[blocks[0][0]])
+    s, e = int(cu[d]), int(cu[d + 1])
+    for j0, n in blocks:
+        assert n > 0 and doc[j0] == d and doc[j0 + n - 1] == d, "blocks lie inside one document"
+    first = min(j0 for j0, _ in blocks)
+    dK = [np.zeros((n, len(kv_heads), q.shape[2])) for _, n in blocks]
+    dV = [np.zeros((n, len(kv_heads), v.shape[2])) for _, n in blocks]
+    for b, g in enumerate(kv_heads):
+        kd, vd = t64(k[s:e, g]), t64(v[s:e, g])
+        for h in range(g * group, (g + 1) * group):
+            qh, doh = t64(q[first:e, h]), t64(do[first:e, h])
+            for i0 in range(first, e, ROW_BLOCK):
+                i1 = min(e, i0 + ROW_BLOCK)
+                qb, dob = qh[i0 - first:i1 - first], doh[i0 - first:i1 - first]
+                S = qb @ kd[:i1 - s].T                                 # keys s .. i1-1
+                S.mul_(scale)
+                # the causal mask: key j > row i is invisible (only keys >= i0 can be)
+                rows = torch.arange(i0, i1)[:, None]
+                cols = torch.arange(i0, i1)[None, :]
+                S[:, i0 - s:].masked_fill_(cols > rows, float("-inf"))
+                mx = S.amax(dim=1, keepdim=True)
+                S.sub_(mx).exp_()                                      # E = exp(S - max)
+                l = S.sum(dim=1)                                       # P = E / l = exp(S - lse)
+                delta = (dob * (S @ vd[:i1 - s])).sum(dim=1) / l       # dO_i . O_i, O = P V
+                for a, (j0, n) in enumerate(blocks):
+                    j1 = min(j0 + n, i1)
+                    if j1 <= j0:
+                        continue
+                    Pb = S[:, j0 - s:j1 - s] / l[:, None]
+                    dPb = dob @ vd[j0 - s:j1 - s].T
+                    dSb = Pb * (dPb - delta[:, None])
+                    dV[a][:j1 - j0, b] += (Pb.T @ dob).numpy()
+                    dK[a][:j1 - j0, b] += scale * (dSb.T @ qb).numpy()
+    return dK, dV
+
+
 # ----------------------------------------------------------------------------
 # Brute-force forms used only to pin the definition above on tiny inputs.
 # ----------------------------------------------------------------------------

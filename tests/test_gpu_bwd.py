@@ -62,18 +62,27 @@ def test_bwd_degenerate_layouts(lens, cp):
     assert_bf16_close(dv, wv, "dV")
 
 
-def test_bwd_long_context_workload_sampled():
-    """T=131072, cp=16, GQA 64/8: dQ at sampled rows, dK/dV at sampled keys (keys near
-    the end of their document, where the oracle's cost per key is small), and two
-    identities over all keys: sum_j dV_j = sum_i sum_{h in g} dO_ih and sum_j dK_j = 0."""
+@pytest.fixture(scope="module")
+def long_context_run():
+    """The long-context workload (T=131072, cp=16, GQA 64/8) through fwd + bwd once."""
     w = syn.WORKLOADS[5]
     cu, (q, k, v, do) = syn.workload_inputs(5, 0)
-    scale = 1 / math.sqrt(128)
     (dq, dk, dv), plan = run_fwd_bwd(cu, w.cp, q, k, v, do)
+    return w, cu, (q, k, v, do), (dq, dk, dv)
+
+
+def test_bwd_long_context_workload_sampled(long_context_run):
+    """dQ at sampled rows (the deepest rows of the 65536-token document among them),
+    dK/dV at sampled keys near the end of their document, and two identities over all
+    keys: sum_j dV_j = sum_i sum_{h in g} dO_ih and sum_j dK_j = 0."""
+    w, cu, (q, k, v, do), (dq, dk, dv) = long_context_run
+    scale = 1 / math.sqrt(128)
     assert np.isfinite(dq).all() and np.isfinite(dk).all() and np.isfinite(dv).all()
     rng = np.random.default_rng(5)
-    # dQ rows: tail of the long document and rows of short documents
-    rows = [65535, 65534, 65400] + [int(x) for x in rng.integers(65536, w.T, 24)]
+    # dQ rows: the long document's first and last tiles, its chunk seams and its deep
+    # rows (walks of up to 512 key tiles), and rows of short documents
+    rows = [0, 127, 128, 2047, 2048, 32768, 49152, 65400, 65534, 65535]
+    rows += [int(x) for x in rng.integers(0, 65536, 6)] + [int(x) for x in rng.integers(65536, w.T, 18)]
     heads = [0, 9, 63]
     want = A.attention_bwd_rows(q, k, v, do, cu, scale, rows, heads)
     assert_bf16_close(dq[rows][:, heads], want, "dQ rows")
@@ -95,6 +104,48 @@ def test_bwd_long_context_workload_sampled():
     walk_k = np.sqrt((dk64 ** 2).sum(axis=0))
     assert np.all(np.abs(dv64.sum(axis=0) - do64.sum(axis=0)) <= 0.02 * walk_v)
     assert np.all(np.abs(dk64.sum(axis=0)) <= 0.05 * walk_k)
+
+
+def test_bwd_long_context_longest_key_tiles_full(long_context_run):
+    """Element by element, the key tiles whose dK/dV walks are the longest of the
+    launch: keys 0..127 of the 65536-token document (seen by all its 512 query tiles x 8
+    query heads) and keys 32768..32895 (256 query tiles), for two key/value heads, with
+    the oracle's blocked key form (every query row of the document that sees them)."""
+    w, cu, (q, k, v, do), (dq, dk, dv) = long_context_run
+    blocks = [(0, 128), (32768, 128)]
+    kvh = [0, 5]
+    wk, wv = A.attention_bwd_key_blocks(q, k, v, do, cu, 1 / math.sqrt(128), blocks, kvh)
+    for (j0, n), gk, gv in zip(blocks, wk, wv):
+        assert_bf16_close(dk[j0:j0 + n][:, kvh], gk, f"dK keys {j0}..{j0 + n - 1}")
+        assert_bf16_close(dv[j0:j0 + n][:, kvh], gv, f"dV keys {j0}..{j0 + n - 1}")
+
+
+def test_bwd_single_16k_document_full():
+    """One 16384-token document, cp=16, GQA 16/2: walks of up to 128 query tiles per key
+    tile and 128 key tiles per query tile, every output compared (O, lse, dQ, dK, dV)."""
+    cu = np.array([0, 16384], dtype=np.int32)
+    q, k, v, do = syn.make_tensors(16384, 16, 2, 128, 128, torch.bfloat16, seed=16, with_do=True)
+    dev = torch.device("cuda:0")
+    plan = thd.Plan(cu, 16).upload()
+    q_rm = thd.thd_kv_gather(plan, q.to(dev))
+    k_rm, v_rm = thd.thd_kv_gather(plan, k.to(dev), v.to(dev))
+    do_rm = thd.thd_kv_gather(plan, do.to(dev))
+    o_rm, lse_rm = thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm)
+    grads = thd.thd_cp_attn_bwd(plan, q_rm, k_rm, v_rm, o_rm, lse_rm, do_rm)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0, "a bounded wait gave up"
+    q_idx = plan.export()["q_idx"]
+    o = unpermute_rows(o_rm.float().cpu().numpy(), q_idx)
+    lse = unpermute_rows(lse_rm.cpu().numpy().T, q_idx).T
+    dq, dk, dv = (unpermute_rows(x.cpu().numpy(), q_idx) for x in grads)
+    scale = 1 / math.sqrt(128)
+    wo, wl = A.attention_fwd(q, k, v, cu, scale)
+    assert_bf16_close(o, wo, "O")
+    assert np.abs(lse - wl).max() <= 1e-3
+    wq, wk, wv = A.attention_bwd(q, k, v, wo, wl, do, cu, scale)
+    assert_bf16_close(dq, wq, "dQ")
+    assert_bf16_close(dk, wk, "dK")
+    assert_bf16_close(dv, wv, "dV")
 
 
 def test_bwd_key_gradients_are_deterministic():

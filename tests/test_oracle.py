@@ -162,9 +162,20 @@ def test_backward_transpose_and_lpt():
                 assert plan["entries"][e, 0] == plan["qtiles"][kt, 2]
                 seen[e] += 1
         assert np.all(seen == 1)
-        assert sorted(plan["lpt"].tolist()) == list(range(n))
-        nk = plan["qtiles"][plan["lpt"], 8]
-        assert np.all(np.diff(nk) <= 0)
+        # longest-first orders: permutations, lengths non-increasing, equal lengths in
+        # ascending tile index (so that the order is unique)
+        lengths = {"lpt": plan["qtiles"][:, 8], "kt_lpt": np.diff(plan["kt_off"])}
+        for key, ln in lengths.items():
+            order = plan[key]
+            assert sorted(order.tolist()) == list(range(n)), key
+            for a, b in zip(order[:-1], order[1:]):
+                assert ln[a] > ln[b] or (ln[a] == ln[b] and a < b), (key, a, b)
+        # each key tile's list length counts the q-tiles of its document that reach it
+        for kt in range(n):
+            d = plan["qtiles"][kt, 1]
+            kpos_min = int(plan["q_idx"][plan["qtiles"][kt, 2]])
+            reach = sum(1 for qt in range(n) if plan["qtiles"][qt, 1] == d and plan["qtiles"][qt, 7] >= kpos_min)
+            assert lengths["kt_lpt"][kt] == reach
 
 
 # ---------------------------------------------------------------- attention pins
@@ -331,6 +342,26 @@ def test_sampled_forms_match_full_forms():
     dKs, dVs = A.attention_bwd_keys(q, k, v, do, cu, 0.4, keys, [0, 1])
     np.testing.assert_allclose(dKs, dk[keys], atol=1e-12, rtol=0)
     np.testing.assert_allclose(dVs, dv[keys], atol=1e-12, rtol=0)
+
+
+def test_key_block_form_matches_full_form():
+    """The blocked key-block form (row blocks smaller than the document, blocks at the
+    document's start, middle and end, ragged sizes) equals the full backward."""
+    cu = np.array([0, 24, 1224, 1300])
+    T, hq, hkv, d = 1300, 4, 2, 8
+    q, k, v, do = (x.numpy() for x in _rand(T, hq, hkv, d, d, 9))
+    o, lse = A.attention_fwd(q, k, v, cu, 0.3)
+    dq, dk, dv = A.attention_bwd(q, k, v, o, lse, do, cu, 0.3)
+    blocks = [(24, 128), (600, 77), (1100, 124)]
+    dKs, dVs = A.attention_bwd_key_blocks(q, k, v, do, cu, 0.3, blocks, [1, 0])
+    for (j0, n), gk, gv in zip(blocks, dKs, dVs):
+        np.testing.assert_allclose(gk, dk[j0:j0 + n][:, [1, 0]], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(gv, dv[j0:j0 + n][:, [1, 0]], atol=1e-12, rtol=0)
+    # a key block in a single-block document, and the last key of a document alone
+    dKs, dVs = A.attention_bwd_key_blocks(q, k, v, do, cu, 0.3, [(0, 24)], [0])
+    np.testing.assert_allclose(dKs[0], dk[0:24][:, [0]], atol=1e-12, rtol=0)
+    dKs, dVs = A.attention_bwd_key_blocks(q, k, v, do, cu, 0.3, [(1299, 1)], [1])
+    np.testing.assert_allclose(dVs[0], dv[1299:1300][:, [1]], atol=1e-12, rtol=0)
 
 
 # ---------------------------------------------------------------- workloads
