@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload forward / K/V-gather measurements")
     ap.add_argument("--clocks-csv", default=None, help="where the nvidia-smi clock samples go (default: a temp file)")
     return ap.parse_args()
 
@@ -84,6 +86,95 @@ def time_plan(thd, cu, cp, reps=5):
         ts.append((time.perf_counter() - t0) * 1e3)
         p.close()
     return statistics.median(ts)
+
+
+def measure_workloads(thd, syn, dev, stream, seed, peaks, iters=10, warmup=3):
+    """Forward attention on the MHA (T=8192), GQA (T=32768) and expanded-MLA (T=65536)
+    workloads, and the K/V-only gather on those and on the long-context workload, each
+    launch timed alone with CUDA events after an L2 flush (a 256 MB write), so that no
+    input is served from L2 left warm by the previous launch.  Returns one sub-object per
+    workload."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        ms = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(a.elapsed_time(b))
+        return statistics.median(ms)
+
+    out = {}
+    for cfg in (2, 3, 4, 5):
+        w = syn.WORKLOADS[cfg]
+        cu = syn.cu_seqlens_of(syn.doc_lengths(cfg, seed))
+        plan = thd.Plan(cu, w.cp).upload()
+        g = torch.Generator(device=dev).manual_seed(seed + 1)
+        k = torch.randn(w.T, w.hkv, w.dqk, device=dev, generator=g).to(torch.bfloat16)
+        v = (torch.randn(w.T, w.hkv, w.dv, device=dev, generator=g) * w.v_std).to(torch.bfloat16)
+        k_rm, v_rm = torch.empty_like(k), torch.empty_like(v)
+        gather_ms = timed(lambda: thd.thd_kv_gather(plan, k, v, k_rm=k_rm, v_rm=v_rm))
+        gather_bytes = 2 * w.T * w.hkv * (w.dqk + w.dv) * 2 + 4 * w.T
+        gbs = gather_bytes / (gather_ms / 1e3) / 1e9
+        rec = {"workload": (f"{w.name}: cp={w.cp}, T={w.T}, {len(cu) - 1} docs, heads {w.hq}/{w.hkv}, "
+                            f"head dims {w.dqk}/{w.dv}, bf16, seed {seed}"),
+               "kv_gather": {"ms": gather_ms, "gbs": gbs, "frac_of_hbm": gbs / hbm, "bytes": gather_bytes,
+                             "l2": "flushed before each launch"}}
+        if cfg != 5:
+            q = torch.randn(w.T, w.hq, w.dqk, device=dev, generator=g).to(torch.bfloat16)
+            q_rm = thd.thd_kv_gather(plan, q)
+            o_rm = torch.empty(w.T, w.hq, w.dv, dtype=torch.bfloat16, device=dev)
+            lse_rm = torch.empty(w.hq, w.T, dtype=torch.float32, device=dev)
+            fwd_ms = timed(lambda: thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm))
+            flops = plan.causal_pairs * w.hq * 2 * (w.dqk + w.dv)
+            tile_flops = plan.n_entries * 128 * 128 * w.hq * 2 * (w.dqk + w.dv)
+            tf = flops / (fwd_ms / 1e3) / 1e12
+            rec["fwd"] = {"ms": fwd_ms, "tflops": tf, "frac_of_peak": tf / burst, "flops": flops,
+                          "density_ceiling": flops / tile_flops,
+                          "tile_tflops": tile_flops / (fwd_ms / 1e3) / 1e12,
+                          "peak_source": "bf16_tflops (burst: the launch is timed alone)",
+                          "l2": "flushed before each launch"}
+            del q, q_rm, o_rm, lse_rm
+        torch.cuda.synchronize(dev)
+        if plan.device_status() != 0:
+            raise RuntimeError(f"a kernel's bounded wait gave up on {w.name}")
+        out[w.name] = rec
+        plan.close()
+        del k, v, k_rm, v_rm
+    del flush
+    return out
+
+
+def measure_replan(thd, syn, plan, dev, stream, seed, w):
+    """Re-planning for a new batch: thd_cp_plan_update of an uploaded plan with another
+    long-context layout (seed + 1), then back.  host_ms is the wall time of the call
+    (partition and tables built on the host, copied into pinned staging, copy enqueued);
+    copy_ms is the device time of its table copy on the stream."""
+    import torch
+    res = []
+    for s_ in (seed + 1, seed):
+        cu = syn.cu_seqlens_of(syn.doc_lengths(WORKLOAD, s_))
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        a.record(stream)
+        plan.update(cu, w.cp, stream=stream)
+        b.record(stream)
+        host_ms = (time.perf_counter() - t0) * 1e3
+        torch.cuda.synchronize(dev)
+        res.append({"seed": s_, "host_ms": host_ms, "copy_ms": a.elapsed_time(b), "n_docs": len(cu) - 1,
+                    "n_entries": plan.n_entries})
+    return {"new_layout": res[0], "back": res[1],
+            "note": "thd_cp_plan_update on the uploaded plan: no device-wide synchronisation"}
 
 
 def flop_counts(pairs, w):
@@ -430,6 +521,13 @@ def run_native(args):
     rope_bytes = 2 * T * w.hq * w.dqk * 2 + T * (w.dqk // 2) * 8 * 2 + 4 * T
     del q_rope, rope_ws
 
+    # ------------------------------------------------ re-plan for a new layout, other workloads
+    peaks, peak_src = load_peaks()
+    replan = measure_replan(thd, syn, plan, dev, stream, args.seed, w)
+    workloads = None
+    if not args.no_workloads:
+        workloads = measure_workloads(thd, syn, dev, stream, args.seed, peaks)
+
     # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1)
     cpu = None
     if info.rank == 0 and info.world == 1 and not args.no_cpu_baseline:
@@ -440,7 +538,6 @@ def run_native(args):
                "sample": (f"oracle fwd+bwd (fp64 numpy) on the {len(cu_s) - 1} short documents "
                           f"({int(cu_s[-1])} tokens) x {n_heads} query heads, {dt:.1f} s")}
 
-    peaks, peak_src = load_peaks()
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     bwd_tf = bwd_fl / (bwd_ms / 1e3) / 1e12
@@ -466,7 +563,9 @@ def run_native(args):
                  "frac_of_hbm": rope_bytes / (rope_ms / 1e3) / 1e9 / hbm, "bytes": rope_bytes,
                  "note": "thd_rope_apply on Q with per-document positions, outside the timed step"},
         "plan": {"host_ms": plan_host_ms, "upload_ms": plan_upload_ms, "q_tiles": plan.n_qtiles,
-                 "note": "thd_cp_plan + thd_cp_plan_upload, once per layout (cached), outside the timed step"},
+                 "note": "thd_cp_plan + thd_cp_plan_upload, once per layout (cached), outside the timed step",
+                 "replan": replan},
+        "workloads": workloads,
         "gather": {"ms": gather_ms, "gbs": gather_gbs, "frac_of_hbm": gather_gbs / hbm, "bytes": gather_bytes,
                    "hbm_peak_gbs": hbm, "peak_source": peak_src},
         "e2e": e2e,
