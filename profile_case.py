@@ -3,18 +3,21 @@ benchmarked workload (one long document of T/2 tokens plus lognormal(512, 1)
 documents in multiples of 32, GQA 64/8, head dim 128, cp=16) at a size whose
 inputs still exceed L2 but fit a profiler's replay budget.
 
-    python -m context_packed_sequence_cp_b200.profile_case [--T 16384] [--iters 2]
+    python profile_case.py [--T 16384] [--iters 2]
 
 Each iteration launches gather (Q, K/V, dO), forward and backward once.
 """
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import numpy as np
 import torch
 
-import context_packed_sequence_cp_b200 as thd
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+import context_packed_sequence_cp_b200 as thd  # noqa: E402
 
 
 def layout(T: int, seed: int) -> np.ndarray:
