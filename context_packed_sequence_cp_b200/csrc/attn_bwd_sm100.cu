@@ -28,6 +28,8 @@
 // kernel that reduces partial dQ tiles into global memory, but the reductions of
 // the single kernel move 64 KB per (query tile, key tile, head) through L2 and cap
 // at the L2's reduction bandwidth once dQ outgrows L2.
+#include <cstdlib>
+
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -82,7 +84,8 @@ __device__ __forceinline__ int visible_keys(int qpos, int nvalid, int kpos0, int
 // ---------------------------------------------------------------- prep
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
-                                                       float* __restrict__ delta, int64_t rows, int hq, int64_t T) {
+                                                       float* __restrict__ delta, float* __restrict__ dq_zero,
+                                                       int64_t rows, int hq, int64_t T) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * 8;
     for (int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); w < rows; w += nwarps) {
@@ -101,6 +104,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) delta[(int64_t)(w % hq) * T + w / hq] = s;
+        // the fused kernel accumulates dQ with reductions: its rows start at zero
+        if (dq_zero) *reinterpret_cast<float4*>(dq_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -654,18 +659,434 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+
+// ================================================================ fused dK / dV / dQ
+// One CTA per (key tile, key/value head g), walked like dkdv_kernel, and in the same
+// walk dQ: per step (query tile, query head)
+//   a  S^T  = K Q^T          -> TMEM X        b  dP^T = V dO^T -> TMEM Y
+//   P^T = exp(S^T - lse) as bf16 over S^T (X); dS^T = P^T (dP^T - Delta) as bf16 into
+//   shared memory (128-byte swizzled, the layout of a [key][query] tile)
+//   c  dV += P^T dO   (A from TMEM X)
+//   d  dK += dS^T Q   (A = dS^T from shared memory, K-major)
+//   e  Y   = dS K     (A = dS from the same bytes read MN-major: this CTA's share of
+//                      the query tile's dQ), drained by the compute warps and added
+//                      into the fp32 dQ with vector reductions at L2
+// issued as c(i), a(i+1), d(i), e(i), b(i+1).  No tile is computed twice.
+struct FusedLayout {
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kTile;
+    static constexpr int kOffQ = kOffV + kTile;             // 2 stages
+    static constexpr int kOffDO = kOffQ + 2 * kTile;        // 2 stages
+    static constexpr int kOffDS = kOffDO + 2 * kTile;       // dS^T, bf16 [128 keys][128 queries]
+    static constexpr int kOffStat = kOffDS + kTile;         // per dO stage: lse2[128], delta[128]
+    static constexpr int kOffBar = kOffStat + 2 * 256 * 4;
+    static constexpr int kBytes = kOffBar + 256;
+    static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+// Phases: every barrier is used once per step (or per stage use) and its next phase
+// needs work that its waiter has not released yet, so parities are unambiguous:
+//   s_full   commit after a(i)   (waited: compute P1(i); producer before dO(i+1): c(i-1) done)
+//   dp_full  commit after b(i)   (compute P2(i))
+//   dq_full  commit after e(i)   (compute drain of dQ(i); producer before Q(i+2): d(i) done)
+//   p_ready / ds_ready / dq_free  arrivals of the 256 compute threads (issuer)
+struct FusedBars {
+    uint64_t kv_full, q_full[2], do_full[2], stat_free[2], s_full, dp_full, dq_full, p_ready, ds_ready, dq_free,
+        acc_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
+    using L = FusedLayout;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    FusedBars* bars = reinterpret_cast<FusedBars*>(smem_raw + L::kOffBar);
+    float* s_stat = reinterpret_cast<float*>(smem_raw + L::kOffStat);
+    const uint32_t sK = base + L::kOffK, sV = base + L::kOffV, sQ = base + L::kOffQ, sDO = base + L::kOffDO;
+    const uint32_t sDS = base + L::kOffDS;
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int group = a.hq / a.hkv;
+    const int n_kt = (int)(gridDim.x / (unsigned)a.hkv);
+    const int kt = a.kt_lpt[blockIdx.x % n_kt];
+    const int g = blockIdx.x / n_kt;
+    const int* KT = a.qtiles + (size_t)kt * 12;
+    const int k0 = KT[2], kn = KT[3];
+    const int l0 = a.kt_off[kt], llen = a.kt_off[kt + 1] - l0;
+    const int n_it = group * llen;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->kv_full), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&bars->q_full[s]), 1);
+            mbar_init(smem_u32(&bars->do_full[s]), 1 + 32);      // expect_tx + the warp's lse/Delta stores
+            mbar_init(smem_u32(&bars->stat_free[s]), kCompute);  // lse/Delta of the stage read by every thread
+        }
+        mbar_init(smem_u32(&bars->s_full), 1);
+        mbar_init(smem_u32(&bars->dp_full), 1);
+        mbar_init(smem_u32(&bars->dq_full), 1);
+        mbar_init(smem_u32(&bars->p_ready), kCompute);
+        mbar_init(smem_u32(&bars->ds_ready), kCompute);
+        mbar_init(smem_u32(&bars->dq_free), kCompute);
+        mbar_init(smem_u32(&bars->acc_done), 1);
+        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
+        if (base & 1023u) atomicCAS(a.status, 0, 99);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (bars->abort || n_it == 0) return;  // misaligned, or an earlier CTA timed out: do nothing
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t tX = tmem, tY = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
+
+    if (warp == 0) {
+        // ---------------------------------------------------- producer warp
+        const float log2e = 1.4426950408889634f;
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            const uint32_t kvf = smem_u32(&bars->kv_full);
+            mbar_arrive_expect_tx(kvf, 2 * kTile);
+            for (int c = 0; c < 2; ++c) {
+                tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
+                tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
+            }
+        }
+        StepMeta cur = load_meta(a, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        for (int it = 0; it < n_it; ++it) {
+            const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
+            if (hh == 0 && it > 0) {
+                cur = nxt;
+                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+            }
+            const int h = g * group + hh;
+            const int row0 = cur.row0;
+            float lv[4], dv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t row = (int64_t)row0 + lane + 32 * u;
+                lv[u] = row < a.T ? __ldg(a.lse + (int64_t)h * a.T + row) * log2e : 0.f;
+                dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
+            }
+            const int st = it & 1;
+            // dO(it) refills the stage c(it-2) read: c(it-2) is issued before a(it-1).
+            if (it >= 2) {
+                mbar_wait(smem_u32(&bars->s_full), (it - 1) & 1, abort, a.status, 61);
+                mbar_wait(smem_u32(&bars->stat_free[st]), ((it >> 1) - 1) & 1, abort, a.status, 62);
+            }
+            const uint32_t f = smem_u32(&bars->do_full[st]);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(f, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
+            }
+            float* stat = s_stat + st * 256;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                stat[lane + 32 * u] = lv[u];
+                stat[128 + lane + 32 * u] = dv[u];
+            }
+            mbar_arrive(f);
+            // Q(it) refills the stage d(it-2) read: d(it-2) is issued before e(it-2).
+            if (it >= 2) mbar_wait(smem_u32(&bars->dq_full), (it - 2) & 1, abort, a.status, 63);
+            if (lane == 0) {
+                const uint32_t qf = smem_u32(&bars->q_full[st]);
+                mbar_arrive_expect_tx(qf, kTile);
+                for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, qf, c * 64, h, row0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
+            constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);   // A TMEM / K-major, B MN-major
+            constexpr uint32_t idMM = idesc_bf16_f32(128, 128, true, true);    // A and B MN-major
+            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
+            const uint32_t klo = smem_desc_lo(sK, 16), vlo = smem_desc_lo(sV, 16);
+            const uint32_t kmlo = smem_desc_lo(sK, kBox);   // K as the MN-major B of e
+            const uint32_t dslo = smem_desc_lo(sDS, 16);    // dS^T, K-major A of d
+            const uint32_t dsmlo = smem_desc_lo(sDS, kBox); // dS, MN-major A of e
+            auto issue_a = [&](int it) {  // S^T = K Q^T -> X
+                const int st = it & 1;
+                mbar_wait(smem_u32(&bars->q_full[st]), (it >> 1) & 1, abort, a.status, 64);
+                tc_fence_after();
+                const uint32_t qlo = smem_desc_lo(sQ + st * kTile, 16);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(tX, smem_desc_of(klo + off, dhi), smem_desc_of(qlo + off, dhi), idKK, kk > 0);
+                }
+                mma_commit(smem_u32(&bars->s_full));
+            };
+            auto issue_b = [&](int it) {  // dP^T = V dO^T -> Y
+                const int st = it & 1;
+                mbar_wait(smem_u32(&bars->do_full[st]), (it >> 1) & 1, abort, a.status, 65);
+                tc_fence_after();
+                const uint32_t dlo = smem_desc_lo(sDO + st * kTile, 16);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(tY, smem_desc_of(vlo + off, dhi), smem_desc_of(dlo + off, dhi), idKK, kk > 0);
+                }
+                mma_commit(smem_u32(&bars->dp_full));
+            };
+            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 66);
+            tc_fence_after();
+            issue_a(0);
+            issue_b(0);
+            for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
+                // c: dV += P^T dO, once P^T is in X
+                mbar_wait(smem_u32(&bars->p_ready), it & 1, abort, a.status, 67);
+                tc_fence_after();
+                const uint32_t dlo = smem_desc_lo(sDO + st * kTile, kBox);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tDV, tX + kk * 8, smem_desc_of(dlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
+                // a of the next step: X is rewritten only after c has read it (issue order)
+                if (it + 1 < n_it) issue_a(it + 1);
+                // d: dK += dS^T Q and e: Y = dS K, once dS^T is in shared memory
+                mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 68);
+                tc_fence_after();
+                const uint32_t qlo = smem_desc_lo(sQ + st * kTile, kBox);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    mma_ss(tDK, smem_desc_of(dslo + off, dhi), smem_desc_of(qlo + kk * (2048 >> 4), dhi), idTM,
+                           (it > 0 || kk > 0));
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tY, smem_desc_of(dsmlo + kk * (2048 >> 4), dhi), smem_desc_of(kmlo + kk * (2048 >> 4), dhi),
+                           idMM, kk > 0);
+                mma_commit(smem_u32(&bars->dq_full));
+                // b of the next step: Y is rewritten only after dQ(it) has been read out
+                if (it + 1 < n_it) {
+                    mbar_wait(smem_u32(&bars->dq_free), it & 1, abort, a.status, 69);
+                    issue_b(it + 1);
+                }
+            }
+            mma_commit(smem_u32(&bars->acc_done));
+        }
+    } else {
+        // ---------------------------------------------------- compute warpgroups
+        const int ct = threadIdx.x - 64;         // 0..255
+        const int hf = ct >> 7;                  // column half
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;            // TMEM lane: key row (X, Y as S^T / dP^T), query row (Y as dQ)
+        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const float sl2 = a.scale_log2;
+        const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
+        // this thread's 128-byte row of dS^T: box hf, row r, 16-byte chunks swizzled by r % 8
+        const uint32_t ds_row = sDS + hf * kBox + r * 128;
+        StepMeta cur = load_meta(a, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        StepMeta prev = cur;  // the step whose dQ is drained
+        int prev_h = 0;
+        // dQ(it) = dS K of this key tile, rows = the step's query rows: read out of Y
+        // (which is then released for b(it+1)), and added, times scale, into the global
+        // fp32 accumulator.  A warp holds 32 query rows x 64 columns; it transposes them
+        // through its own 4 KB of the dS^T buffer (the rows it alone writes, free once
+        // e(it) has retired) so that every vector reduction instruction covers 4 whole
+        // 128-byte row segments instead of 32 scattered 16-byte pieces.
+        const uint32_t warp_stage = sDS + hf * kBox + wq * 32 * 128;
+        auto drain = [&](int it, const StepMeta& mt, int h) {
+            mbar_wait(smem_u32(&bars->dq_full), it & 1, abort, a.status, 70);
+            tc_fence_after();
+            const float sc = a.scale;
+            const int sub = lane >> 3, chunk = lane & 7;     // reader: row 4j + sub, 16-byte chunk
+            uint32_t v[32];
+            auto stage = [&]() {  // this lane's 128-byte row segment, chunks swizzled by lane % 8
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(warp_stage + lane * 128 + ((c ^ (lane & 7)) << 4),
+                                 __float_as_uint(__uint_as_float(v[4 * c]) * sc),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 1]) * sc),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 2]) * sc),
+                                 __float_as_uint(__uint_as_float(v[4 * c + 3]) * sc));
+            };
+            auto reduce = [&](int k) {  // 8 instructions, each 4 rows x 128 contiguous bytes
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int rr = 4 * j + sub;                // row within the warp's 32
+                    const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+                    const int q = wq * 32 + rr;                // query row of the tile
+                    if (q < mt.m)
+                        red_add_v4(a.dq_acc + ((int64_t)(mt.row0 + q) * a.hq + h) * kD + hf * 64 + 32 * k + 4 * chunk,
+                                   x.x, x.y, x.z, x.w);
+                }
+            };
+            tmem_ld32(tY + lane_addr + hf * 64, v);
+            tmem_wait_ld();
+            stage();
+            tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
+            __syncwarp();
+            reduce(0);
+            __syncwarp();
+            stage();
+            __syncwarp();
+            reduce(1);
+            __syncwarp();
+        };
+        for (int it = 0; it < n_it; ++it) {
+            const int st = it & 1;
+            const int pos = it / group, hh = it - pos * group;
+            if (hh == 0 && it > 0) {
+                cur = nxt;
+                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+            }
+            const int m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
+            // visible query columns of this key row: a suffix [lo, hi) of the tile
+            int lo = 0, hi = m;
+            if (r >= cur.nvalid) hi = 0;
+            else if (cur.cls != 2) {
+                const int n1 = min(qbrk, m);
+                if (kpos_r <= qpos0) lo = 0;
+                else if (kpos_r - qpos0 < n1) lo = kpos_r - qpos0;
+                else {
+                    const int p1 = qpos0 + qbrk + qjump;   // position of row qbrk
+                    lo = (kpos_r <= p1) ? n1 : min(m, n1 + (kpos_r - p1));
+                }
+            }
+            const float* stat = s_stat + st * 256;
+
+            // ---- P1: P^T = exp(S^T - lse) on this thread's 64 query columns, bf16 over S^T
+            mbar_wait(smem_u32(&bars->do_full[st]), (it >> 1) & 1, abort, a.status, 71);  // lse/Delta staged
+            mbar_wait(smem_u32(&bars->s_full), it & 1, abort, a.status, 72);
+            tc_fence_after();
+            float p[64];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t sv[32];
+                const int c0 = hf * 64 + ch * 32;
+                tmem_ld32(tX + lane_addr + c0, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int t = 0; t < 32; t += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(stat + c0 + t);
+                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = c0 + t + u;
+                        const float e = ex2(fmaf(__uint_as_float(sv[t + u]), sl2, -lq[u]));
+                        p[ch * 32 + t + u] = (i >= lo && i < hi) ? e : 0.f;
+                    }
+                }
+            }
+            named_bar_sync(2 + wq, 64);  // both halves of these rows have read S^T before P^T overwrites it
+            {
+                uint32_t pk[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(p[2 * t], p[2 * t + 1]);
+                tmem_st32(tX + lane_addr + hf * 32, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_ready));
+
+            // ---- drain dQ of the previous step (frees Y for b(it), and the dS^T buffer)
+            if (it >= 1) drain(it - 1, prev, prev_h);
+            prev = cur;
+            prev_h = a.hq / a.hkv * g + hh;
+
+            // ---- P2: dS^T = P^T (dP^T - Delta) -> shared memory
+            mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 73);
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t dpv[32];
+                const int c0 = hf * 64 + ch * 32;
+                tmem_ld32(tY + lane_addr + c0, dpv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {   // 16-byte chunk (8 queries) ch * 4 + j of this half-row
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int t = j * 8 + 2 * u;
+                        const float2 d2 = *reinterpret_cast<const float2*>(stat + 128 + c0 + t);
+                        w4[u] = pack_bf16x2(p[ch * 32 + t] * (__uint_as_float(dpv[t]) - d2.x),
+                                            p[ch * 32 + t + 1] * (__uint_as_float(dpv[t + 1]) - d2.y));
+                    }
+                    const int chunk = ch * 4 + j;
+                    st_shared_v4(ds_row + ((chunk ^ (r & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            mbar_arrive(smem_u32(&bars->stat_free[st]));  // lse and Delta of this stage read
+            fence_proxy_async_smem();                      // dS^T visible to the tensor pipe
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->ds_ready));
+        }
+        drain(n_it - 1, prev, prev_h);
+        // ---------------------------------------------------- dK, dV epilogue
+        mbar_wait(smem_u32(&bars->acc_done), 0, abort, a.status, 74);
+        tc_fence_after();
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint32_t src = which == 0 ? tDK : tDV;
+            float* out = which == 0 ? a.dk : a.dv;
+            const float mul = which == 0 ? a.scale : 1.f;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t v[32];
+                const int c0 = hf * 64 + ch * 32;
+                tmem_ld32(src + lane_addr + c0, v);
+                tmem_wait_ld();
+                if (r < kn) {
+                    float4* dst = reinterpret_cast<float4*>(out + ((int64_t)(k0 + r) * a.hkv + g) * kD + c0);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        dst[t] = make_float4(__uint_as_float(v[4 * t]) * mul, __uint_as_float(v[4 * t + 1]) * mul,
+                                             __uint_as_float(v[4 * t + 2]) * mul, __uint_as_float(v[4 * t + 3]) * mul);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
 }  // namespace
 
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
+    static const bool fused = [] {
+        const char* e = getenv("THD_BWD_FUSED");
+        return e && e[0] == '1';
+    }();
+    const unsigned kv_grid = (unsigned)((int64_t)n_tiles * a.hkv);
+    if (fused) {
+        static std::atomic<uint64_t> fused_configured{0};
+        if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, fused_configured)) return -1;
+        bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.T * a.hq, a.hq, a.T);
+        if (cudaGetLastError() != cudaSuccess) return -1;
+        bwd_fused_kernel<<<kv_grid, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, a);
+        return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    }
     static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};
     if (!ensure_dynamic_smem(dkdv_kernel, DkdvLayout::kBytes, dkdv_configured) ||
         !ensure_dynamic_smem(dq_kernel, DqLayout::kBytes, dq_configured))
         return -1;
-    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.T * a.hq, a.hq, a.T);
+    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, nullptr, a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
-    dkdv_kernel<<<(unsigned)((int64_t)n_tiles * a.hkv), kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);
+    dkdv_kernel<<<kv_grid, kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);
     if (cudaGetLastError() != cudaSuccess) return -1;
     dq_kernel<<<(unsigned)((int64_t)n_tiles * a.hq), kThreads, DqLayout::kBytes, stream>>>(q, k, v, dout, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;

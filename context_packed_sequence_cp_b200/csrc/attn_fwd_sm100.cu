@@ -7,8 +7,8 @@
 // and expanded MLA.  Section "Does this PR introduce any user-facing change?":
 // causal attention with EOD reset.
 //
-// One CTA computes one (query tile, query head) work item, items taken in
-// longest-first order.  Warp roles (384 threads):
+// One CTA computes one (query tile, query head) work item; items are ordered by
+// key/value group, then longest-first, then query head.  Warp roles (384 threads):
 //   warp 0      TMA producer of the Q tile and of K of every listed entry;
 //   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
 //               boxes of 64 columns); a stage is refilled once the MMA that read
@@ -111,10 +111,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     volatile int* abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int item = blockIdx.x;
-    const int qt = a.lpt[item / a.hq];
-    const int h = item % a.hq;
-    const int g = h / (a.hq / a.hkv);
+    // Items: key/value groups outermost, then query tiles longest-first, then the query
+    // heads of the group, so that the CTAs resident together walk the K/V tiles of one
+    // group (a working set that stays in L2) instead of all groups at once.
+    const int group = a.hq / a.hkv;
+    const int per_group = (int)(gridDim.x / (unsigned)a.hkv);   // query tiles x group
+    const int g = blockIdx.x / per_group;
+    const int rem = blockIdx.x - g * per_group;
+    const int qt = a.lpt[rem / group];
+    const int h = g * group + rem % group;
     const int* Q = a.qtiles + (size_t)qt * 12;
     const int row0 = Q[2], m = Q[3], qpos0 = Q[4], qbrk = Q[5], qjump = Q[6];
     const int nk = Q[8], e0 = Q[9];
