@@ -699,7 +699,8 @@ struct FusedBars {
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                 const __grid_constant__ CUtensorMap tmDQ, BwdArgs a) {
     using L = FusedLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -757,6 +758,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
+            tma_prefetch_desc(&tmDQ);
             const uint32_t kvf = smem_u32(&bars->kv_full);
             mbar_arrive_expect_tx(kvf, 2 * kTile);
             for (int c = 0; c < 2; ++c) {
@@ -896,17 +898,19 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         StepMeta prev = cur;  // the step whose dQ is drained
         int prev_h = 0;
         // dQ(it) = dS K of this key tile, rows = the step's query rows: read out of Y
-        // (which is then released for b(it+1)), and added, times scale, into the global
-        // fp32 accumulator.  A warp holds 32 query rows x 64 columns; it transposes them
-        // through its own 4 KB of the dS^T buffer (the rows it alone writes, free once
-        // e(it) has retired) so that every vector reduction instruction covers 4 whole
-        // 128-byte row segments instead of 32 scattered 16-byte pieces.
+        // (which is then released for b(it+1)) and added, times scale, into the global
+        // fp32 accumulator.  A warp holds 32 query rows x 64 columns.  It writes them, 32
+        // columns at a time, into its own 4 KB of the dS^T buffer (the rows only it writes,
+        // free once e(it) has retired) in the 128-byte swizzled layout of a 32 x 32 fp32
+        // box, and one lane adds the box into dQ with a TMA tensor reduction (whole 128-byte
+        // row segments).  A warp whose rows run past the query tile (its last, short tile)
+        // adds its valid rows with vector reductions instead.
         const uint32_t warp_stage = sDS + hf * kBox + wq * 32 * 128;
         auto drain = [&](int it, const StepMeta& mt, int h) {
             mbar_wait(smem_u32(&bars->dq_full), it & 1, abort, a.status, 70);
             tc_fence_after();
             const float sc = a.scale;
-            const int sub = lane >> 3, chunk = lane & 7;     // reader: row 4j + sub, 16-byte chunk
+            const bool whole = wq * 32 + 32 <= mt.m;
             uint32_t v[32];
             auto stage = [&]() {  // this lane's 128-byte row segment, chunks swizzled by lane % 8
 #pragma unroll
@@ -917,15 +921,31 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                  __float_as_uint(__uint_as_float(v[4 * c + 2]) * sc),
                                  __float_as_uint(__uint_as_float(v[4 * c + 3]) * sc));
             };
-            auto reduce = [&](int k) {  // 8 instructions, each 4 rows x 128 contiguous bytes
+            auto reduce = [&](int k) {
+                const int col = hf * 64 + 32 * k;
+                if (whole) {
+                    fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_3d(&tmDQ, warp_stage, col, h, mt.row0 + wq * 32);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();   // the box has been read: the rows may be rewritten
+                    }
+                    __syncwarp();
+                } else {
+                    __syncwarp();
+                    const int sub = lane >> 3, chunk = lane & 7;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int rr = 4 * j + sub;                // row within the warp's 32
-                    const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
-                    const int q = wq * 32 + rr;                // query row of the tile
-                    if (q < mt.m)
-                        red_add_v4(a.dq_acc + ((int64_t)(mt.row0 + q) * a.hq + h) * kD + hf * 64 + 32 * k + 4 * chunk,
-                                   x.x, x.y, x.z, x.w);
+                    for (int j = 0; j < 8; ++j) {
+                        const int rr = 4 * j + sub;
+                        const int q = wq * 32 + rr;
+                        if (q < mt.m) {
+                            const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+                            red_add_v4(a.dq_acc + ((int64_t)(mt.row0 + q) * a.hq + h) * kD + col + 4 * chunk, x.x,
+                                       x.y, x.z, x.w);
+                        }
+                    }
+                    __syncwarp();
                 }
             };
             tmem_ld32(tY + lane_addr + hf * 64, v);
@@ -935,13 +955,9 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
-            __syncwarp();
             reduce(0);
-            __syncwarp();
             stage();
-            __syncwarp();
             reduce(1);
-            __syncwarp();
         };
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
@@ -1068,8 +1084,8 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
                      const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
     static const bool fused = [] {
-        const char* e = getenv("THD_BWD_FUSED");
-        return e && e[0] == '1';
+        const char* e = getenv("THD_BWD_SPLIT");
+        return !(e && e[0] == '1');
     }();
     const unsigned kv_grid = (unsigned)((int64_t)n_tiles * a.hkv);
     if (fused) {
@@ -1077,7 +1093,9 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
         if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, fused_configured)) return -1;
         bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.T * a.hq, a.hq, a.T);
         if (cudaGetLastError() != cudaSuccess) return -1;
-        bwd_fused_kernel<<<kv_grid, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, a);
+        CUtensorMap mdq;
+        if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD)) return -1;
+        bwd_fused_kernel<<<kv_grid, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, a);
         return cudaGetLastError() == cudaSuccess ? 0 : -1;
     }
     static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};

@@ -27,6 +27,9 @@ inline bool ensure_dynamic_smem(Kernel* fn, int bytes, std::atomic<uint64_t>& do
 // 128-row boxes and 128-byte swizzle (the layout the tcgen05 descriptors expect).
 // False when the driver's encoder is unavailable or rejects the map.
 bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
+// [rows, heads, dim] fp32 tensor viewed as a 3-D TMA map with 32-column x 1-head x 32-row
+// boxes (128-byte rows) and 128-byte swizzle: the target of tiled reductions.
+bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
 
 // ---- row gather (all-gather layout, and its inverse) -----------------------
 // dst_t[j] = src_t[idx[j]] for whole rows of row_bytes_t bytes, t = 0, 1 (the second
