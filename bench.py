@@ -136,7 +136,9 @@ def measure_workloads(thd, syn, dev, stream, seed, peaks, iters=10, warmup=3):
             lse_rm = torch.empty(w.hq, w.T, dtype=torch.float32, device=dev)
             fwd_ms = timed(lambda: thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm))
             flops = plan.causal_pairs * w.hq * 2 * (w.dqk + w.dv)
-            tile_flops = plan.n_entries * 128 * 128 * w.hq * 2 * (w.dqk + w.dv)
+            # 128 x 128 tile pairs the forward computes (its own tables: rank-major tiles,
+            # position tiles for short-chunk documents)
+            tile_flops = plan.n_fentries * 128 * 128 * w.hq * 2 * (w.dqk + w.dv)
             tf = flops / (fwd_ms / 1e3) / 1e12
             rec["fwd"] = {"ms": fwd_ms, "tflops": tf, "frac_of_peak": tf / burst, "flops": flops,
                           "density_ceiling": flops / tile_flops,

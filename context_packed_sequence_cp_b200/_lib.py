@@ -12,6 +12,7 @@ THD_DTYPE_BF16 = 0
 THD_DTYPE_FP32 = 1
 NOALLOC_MAX_ROWS_X_HEADS = 8388608
 QT_FIELDS = 12
+KSEG = 32
 EN_FIELDS = 8
 
 ERRORS = {
@@ -28,7 +29,8 @@ _F = ctypes.c_float
 SIGNATURES = {
     "thd_cp_plan": (ctypes.c_int, [_PI32, _I32, _I32, ctypes.POINTER(_P)]),
     "thd_cp_plan_info": (ctypes.c_int, [_P, _P]),
-    "thd_cp_plan_export": (ctypes.c_int, [_P, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32]),
+    "thd_cp_plan_export": (ctypes.c_int, [_P, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32]),
+    "thd_cp_plan_export_fwd": (ctypes.c_int, [_P, _PI32, _PI32, _PI32]),
     "thd_cp_plan_upload": (ctypes.c_int, [_P, _P]),
     "thd_cp_plan_update": (ctypes.c_int, [_P, _PI32, _I32, _I32, _P]),
     "thd_cp_plan_destroy": (None, [_P]),
@@ -55,7 +57,8 @@ SIGNATURES = {
 class PlanInfo(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("cp", ctypes.c_int32), ("n_docs", ctypes.c_int32),
                 ("Tl", ctypes.c_int64), ("n_qtiles", ctypes.c_int64), ("n_entries", ctypes.c_int64),
-                ("causal_pairs", ctypes.c_int64)]
+                ("causal_pairs", ctypes.c_int64), ("n_kseg", ctypes.c_int64), ("n_fqtiles", ctypes.c_int64),
+                ("n_fentries", ctypes.c_int64)]
 
 
 class ThdError(RuntimeError):

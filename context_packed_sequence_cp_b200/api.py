@@ -115,10 +115,19 @@ class Plan:
         out = dict(q_idx=np.empty(T, np.int32), rm_of_global=np.empty(T, np.int32),
                    qtiles=np.empty((nq, QT_FIELDS), np.int32), entries=np.empty((ne, EN_FIELDS), np.int32),
                    lpt=np.empty(nq, np.int32), kt_off=np.empty(nq + 1, np.int32),
-                   kt_list=np.empty((ne, 2), np.int32), kt_lpt=np.empty(nq, np.int32))
+                   kt_list=np.empty((ne, 2), np.int32), kt_lpt=np.empty(nq, np.int32),
+                   kt_seg=np.empty(self.n_kseg + 1, np.int32))
         check("thd_cp_plan_export", lib().thd_cp_plan_export(
             self._h, *(_i32p(out[k]) for k in ("q_idx", "rm_of_global", "qtiles", "entries", "lpt",
-                                                "kt_off", "kt_list", "kt_lpt"))))
+                                                "kt_off", "kt_list", "kt_lpt", "kt_seg"))))
+        return out
+
+    def export_fwd(self) -> dict:
+        """The forward tables (thd_cp_plan_export_fwd)."""
+        out = dict(fqtiles=np.empty((self.n_fqtiles, QT_FIELDS), np.int32),
+                   fentries=np.empty((self.n_fentries, EN_FIELDS), np.int32), flpt=np.empty(self.n_fqtiles, np.int32))
+        check("thd_cp_plan_export_fwd", lib().thd_cp_plan_export_fwd(
+            self._h, _i32p(out["fqtiles"]), _i32p(out["fentries"]), _i32p(out["flpt"])))
         return out
 
     def upload(self, stream=None) -> "Plan":
@@ -161,6 +170,8 @@ class Plan:
         self.T, self.cp, self.n_docs = int(info.T), int(info.cp), int(info.n_docs)
         self.Tl, self.n_qtiles, self.n_entries = int(info.Tl), int(info.n_qtiles), int(info.n_entries)
         self.causal_pairs = int(info.causal_pairs)
+        self.n_kseg = int(info.n_kseg)
+        self.n_fqtiles, self.n_fentries = int(info.n_fqtiles), int(info.n_fentries)
 
     def device_status(self, reset: bool = True) -> int:
         v = ctypes.c_int32()

@@ -57,7 +57,8 @@ void free_device(thd_plan* p) {
         p->h_cap[i] = 0;
     }
     p->d_q_idx = p->d_rm_of_global = p->d_qtiles = p->d_entries = p->d_lpt = nullptr;
-    p->d_kt_off = p->d_kt_list = p->d_kt_lpt = p->d_status = nullptr;
+    p->d_kt_off = p->d_kt_list = p->d_kt_lpt = p->d_kt_seg = p->d_status = nullptr;
+    p->d_fqtiles = p->d_fentries = p->d_flpt = nullptr;
     p->uploaded = false;
 }
 
@@ -70,13 +71,16 @@ size_t round_up(size_t n) { return (n + kAlign - 1) & ~(kAlign - 1); }
 // tables outgrow it; the status word at its start survives a re-plan.  Work on `s`
 // enqueued earlier reads the previous tables before the copy overwrites them.
 int copy_tables(thd_plan* p, cudaStream_t s, bool first) {
-    const std::vector<int32_t>* src[] = {&p->q_idx,  &p->rm_of_global, &p->qtiles,  &p->entries,
-                                         &p->lpt,    &p->kt_off,       &p->kt_list, &p->kt_lpt};
-    int32_t** dst[] = {&p->d_q_idx, &p->d_rm_of_global, &p->d_qtiles,  &p->d_entries,
-                       &p->d_lpt,   &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt};
-    size_t off[8];
+    constexpr int kTables = 12;
+    const std::vector<int32_t>* src[kTables] = {&p->q_idx,  &p->rm_of_global, &p->qtiles, &p->entries,
+                                                &p->lpt,    &p->kt_off,       &p->kt_list, &p->kt_lpt,
+                                                &p->kt_seg, &p->fqtiles,      &p->fentries, &p->flpt};
+    int32_t** dst[kTables] = {&p->d_q_idx,  &p->d_rm_of_global, &p->d_qtiles,  &p->d_entries,
+                              &p->d_lpt,    &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt,
+                              &p->d_kt_seg, &p->d_fqtiles,      &p->d_fentries, &p->d_flpt};
+    size_t off[kTables];
     size_t total = kAlign;  // the status word (16 bytes) sits in the first 256
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kTables; ++i) {
         off[i] = total;
         total += round_up(std::max<size_t>(src[i]->size(), 4) * sizeof(int32_t));
     }
@@ -93,7 +97,7 @@ int copy_tables(thd_plan* p, cudaStream_t s, bool first) {
         p->h_cap[st] = cap;
     }
     uint8_t* h = static_cast<uint8_t*>(p->h_stage[st]);
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kTables; ++i)
         if (!src[i]->empty()) std::memcpy(h + off[i], src[i]->data(), src[i]->size() * sizeof(int32_t));
     if (p->d_cap < total) {
         void* fresh = nullptr;
@@ -116,7 +120,7 @@ int copy_tables(thd_plan* p, cudaStream_t s, bool first) {
     if (cudaEventRecord(p->staged[st], s) != cudaSuccess) return THD_ERR_CUDA;
     p->next_stage = st ^ 1;
     p->d_status = reinterpret_cast<int32_t*>(d);
-    for (int i = 0; i < 8; ++i) *dst[i] = reinterpret_cast<int32_t*>(d + off[i]);
+    for (int i = 0; i < kTables; ++i) *dst[i] = reinterpret_cast<int32_t*>(d + off[i]);
     return THD_OK;
 }
 
@@ -156,6 +160,18 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int dim) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)dim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)dim * 2};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -171,6 +187,7 @@ bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int he
 }  // namespace thd
 
 using thd::make_map_bf16;
+using thd::make_map_bf16_rows;
 
 extern "C" {
 
@@ -196,11 +213,15 @@ int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out) {
     out->n_qtiles = plan->n_qtiles();
     out->n_entries = plan->n_entries();
     out->causal_pairs = plan->causal_pairs;
+    out->n_kseg = plan->kt_seg.empty() ? 0 : (int64_t)plan->kt_seg.size() - 1;
+    out->n_fqtiles = plan->n_fqtiles();
+    out->n_fentries = plan->n_fentries();
     return THD_OK;
 }
 
 int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global, int32_t* qtiles,
-                       int32_t* entries, int32_t* lpt, int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt) {
+                       int32_t* entries, int32_t* lpt, int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt,
+                       int32_t* kt_seg) {
     if (!plan) return THD_ERR_INVALID_ARG;
     auto cp = [](int32_t* dst, const std::vector<int32_t>& v) {
         if (dst && !v.empty()) std::memcpy(dst, v.data(), v.size() * sizeof(int32_t));
@@ -213,6 +234,18 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
     cp(kt_off, plan->kt_off);
     cp(kt_list, plan->kt_list);
     cp(kt_lpt, plan->kt_lpt);
+    cp(kt_seg, plan->kt_seg);
+    return THD_OK;
+}
+
+int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt) {
+    if (!plan) return THD_ERR_INVALID_ARG;
+    auto cp = [](int32_t* dst, const std::vector<int32_t>& v) {
+        if (dst && !v.empty()) std::memcpy(dst, v.data(), v.size() * sizeof(int32_t));
+    };
+    cp(fqtiles, plan->fqtiles);
+    cp(fentries, plan->fentries);
+    cp(flpt, plan->flpt);
     return THD_OK;
 }
 
@@ -257,6 +290,10 @@ int thd_cp_plan_update(thd_cp_plan_t plan, const int32_t* cu_seqlens, int32_t n_
     plan->kt_off.swap(fresh.kt_off);
     plan->kt_list.swap(fresh.kt_list);
     plan->kt_lpt.swap(fresh.kt_lpt);
+    plan->kt_seg.swap(fresh.kt_seg);
+    plan->fqtiles.swap(fresh.fqtiles);
+    plan->fentries.swap(fresh.fentries);
+    plan->flpt.swap(fresh.flpt);
     if (!plan->uploaded) return THD_OK;
     // On a failed copy the device tables no longer match the host tables: the plan
     // becomes not-uploaded, and a later thd_cp_plan_upload copies them afresh.
@@ -351,9 +388,10 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
         !make_map_bf16(&mkr, k_rope_rm, plan->T, 1, d_rope) || !make_map_bf16(&mv, v_rm, plan->T, hkv, dv))
         return THD_ERR_CUDA;
     thd::FwdArgs a;
-    a.qtiles = plan->d_qtiles;
+    a.qtiles = plan->d_qtiles;   // rank-major tiles only (position tiles are not built for the compact keys)
     a.entries = plan->d_entries;
     a.lpt = plan->d_lpt;
+    a.rm_of_global = plan->d_rm_of_global;
     a.o = static_cast<__nv_bfloat16*>(o_rm);
     a.lse = lse_rm;
     a.hq = hq;
@@ -378,18 +416,21 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     if (!aligned16(q_rm) || !aligned16(k_rm) || !aligned16(v_rm) || !aligned16(o_rm) || !aligned16(lse_rm))
         return THD_ERR_MISALIGNED;
     const int64_t items = plan->n_qtiles() * (int64_t)hq;
-    if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
+    if (items > INT32_MAX || plan->n_fqtiles() * (int64_t)hq > INT32_MAX) return THD_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == THD_DTYPE_BF16) {
         if (!((dqk == 128 && dv == 128) || (dqk == 192 && dv == 128))) return THD_ERR_UNSUPPORTED;
-        CUtensorMap mq, mk, mv;
+        CUtensorMap mq, mk, mv, mqg, mkg, mvg;
         if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
-            !make_map_bf16(&mv, v_rm, plan->T, hkv, dv))
+            !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, dqk) ||
+            !make_map_bf16_rows(&mkg, k_rm, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
             return THD_ERR_CUDA;
+        // the forward tables: rank-major tiles, position tiles for short-chunk documents
         thd::FwdArgs a;
-        a.qtiles = plan->d_qtiles;
-        a.entries = plan->d_entries;
-        a.lpt = plan->d_lpt;
+        a.qtiles = plan->d_fqtiles;
+        a.entries = plan->d_fentries;
+        a.lpt = plan->d_flpt;
+        a.rm_of_global = plan->d_rm_of_global;
         a.o = static_cast<__nv_bfloat16*>(o_rm);
         a.lse = lse_rm;
         a.hq = hq;
@@ -397,8 +438,9 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
         a.T = plan->T;
         a.scale_log2 = scale * 1.4426950408889634f;
         a.status = plan->d_status;
-        if (items == 0) return THD_OK;
-        return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, a, (int)items, s) ? THD_ERR_CUDA : THD_OK;
+        const int64_t fitems = plan->n_fqtiles() * (int64_t)hq;
+        if (fitems == 0) return THD_OK;
+        return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)fitems, s) ? THD_ERR_CUDA : THD_OK;
     }
     if (dtype == THD_DTYPE_FP32) {
         if (!((dqk == 64 && dv == 64) || (dqk == 128 && dv == 128))) return THD_ERR_UNSUPPORTED;
@@ -461,6 +503,8 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     a.kt_off = plan->d_kt_off;
     a.kt_list = plan->d_kt_list;
     a.kt_lpt = plan->d_kt_lpt;
+    a.kt_seg = plan->d_kt_seg;
+    a.n_kseg = (int32_t)(plan->kt_seg.size() - 1);
     a.o = static_cast<const __nv_bfloat16*>(o_rm);
     a.dout = static_cast<const __nv_bfloat16*>(do_rm);
     a.lse = lse_rm;
@@ -476,7 +520,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     a.status = plan->d_status;
     const int64_t nkt = plan->n_qtiles();
     if (nkt == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, num_sms_current(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, plan->kt_seg.back(), num_sms_current(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

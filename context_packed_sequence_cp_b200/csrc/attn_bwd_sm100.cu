@@ -34,6 +34,7 @@
 
 #include "kernels.h"
 #include "sm100.cuh"
+#include "thdcp.h"
 
 namespace thd {
 namespace {
@@ -85,7 +86,8 @@ __device__ __forceinline__ int visible_keys(int qpos, int nvalid, int kpos0, int
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
                                                        float* __restrict__ delta, float* __restrict__ dq_zero,
-                                                       int64_t rows, int hq, int64_t T) {
+                                                       float* __restrict__ dk_zero, float* __restrict__ dv_zero,
+                                                       int64_t kv_rows, int64_t rows, int hq, int64_t T) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * 8;
     for (int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); w < rows; w += nwarps) {
@@ -104,8 +106,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) delta[(int64_t)(w % hq) * T + w / hq] = s;
-        // the fused kernel accumulates dQ with reductions: its rows start at zero
+        // the fused kernel accumulates dQ, dK and dV with reductions: they start at zero
         if (dq_zero) *reinterpret_cast<float4*>(dq_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dk_zero && w < kv_rows) {
+            *reinterpret_cast<float4*>(dk_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dv_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
 }
 
@@ -700,7 +706,8 @@ struct FusedBars {
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                 const __grid_constant__ CUtensorMap tmDQ, BwdArgs a) {
+                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                 const __grid_constant__ CUtensorMap tmDV, BwdArgs a) {
     using L = FusedLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -712,12 +719,27 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = a.hq / a.hkv;
-    const int n_kt = (int)(gridDim.x / (unsigned)a.hkv);
-    const int kt = a.kt_lpt[blockIdx.x % n_kt];
-    const int g = blockIdx.x / n_kt;
+    // Work item: segment j (list entries j*THD_KSEG ..) of a key tile, for key/value
+    // group g.  Items run groups outermost, then segment, then key tiles longest-first:
+    // the resident CTAs walk the same THD_KSEG query tiles of a document, so the dQ tiles
+    // they add into stay in L2 while they are hot.
+    const int per_group = a.kt_seg[a.n_kseg];
+    const int g = blockIdx.x / per_group;
+    const int item = blockIdx.x - g * per_group;
+    int seg = 0;
+    {
+        int hi = a.n_kseg;  // kt_seg[seg] <= item < kt_seg[hi]
+        while (hi - seg > 1) {
+            const int mid = (seg + hi) >> 1;
+            if (__ldg(a.kt_seg + mid) <= item) seg = mid;
+            else hi = mid;
+        }
+    }
+    const int kt = a.kt_lpt[item - a.kt_seg[seg]];
     const int* KT = a.qtiles + (size_t)kt * 12;
     const int k0 = KT[2], kn = KT[3];
-    const int l0 = a.kt_off[kt], llen = a.kt_off[kt + 1] - l0;
+    const int l0 = a.kt_off[kt] + seg * THD_KSEG;
+    const int llen = min(THD_KSEG, a.kt_off[kt + 1] - l0);
     const int n_it = group * llen;
 
     if (threadIdx.x == 0) {
@@ -759,6 +781,8 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
             tma_prefetch_desc(&tmDQ);
+            tma_prefetch_desc(&tmDK);
+            tma_prefetch_desc(&tmDV);
             const uint32_t kvf = smem_u32(&bars->kv_full);
             mbar_arrive_expect_tx(kvf, 2 * kTile);
             for (int c = 0; c < 2; ++c) {
@@ -897,67 +921,71 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (llen > 1) nxt = load_meta(a, l0 + 1);
         StepMeta prev = cur;  // the step whose dQ is drained
         int prev_h = 0;
-        // dQ(it) = dS K of this key tile, rows = the step's query rows: read out of Y
-        // (which is then released for b(it+1)) and added, times scale, into the global
-        // fp32 accumulator.  A warp holds 32 query rows x 64 columns.  It writes them, 32
-        // columns at a time, into its own 4 KB of the dS^T buffer (the rows only it writes,
-        // free once e(it) has retired) in the 128-byte swizzled layout of a 32 x 32 fp32
-        // box, and one lane adds the box into dQ with a TMA tensor reduction (whole 128-byte
-        // row segments).  A warp whose rows run past the query tile (its last, short tile)
-        // adds its valid rows with vector reductions instead.
+        // Partial sums leave the CTA through its warps: a warp holds 32 rows x 64 columns
+        // of an fp32 TMEM accumulator (rows 32 wq .., columns hf*64 ..).  It writes them, 32
+        // columns at a time, into its own 4 KB of the dS^T buffer (the rows only it writes)
+        // in the 128-byte swizzled layout of a 32 x 32 fp32 box, and one lane adds the box
+        // into global memory with a TMA tensor reduction (whole 128-byte row segments).  A
+        // warp whose rows run past the tile's valid rows adds those with vector reductions.
         const uint32_t warp_stage = sDS + hf * kBox + wq * 32 * 128;
+        auto stage = [&](const uint32_t (&v)[32], float mul) {  // chunks swizzled by lane % 8
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(warp_stage + lane * 128 + ((c ^ (lane & 7)) << 4),
+                             __float_as_uint(__uint_as_float(v[4 * c]) * mul),
+                             __float_as_uint(__uint_as_float(v[4 * c + 1]) * mul),
+                             __float_as_uint(__uint_as_float(v[4 * c + 2]) * mul),
+                             __float_as_uint(__uint_as_float(v[4 * c + 3]) * mul));
+        };
+        // adds the staged box at (row0 + 32 wq, head, col) of a [rows, heads, 128] fp32
+        // tensor with `valid` rows from row0 on
+        // The staging rows are rewritten only after stage_free(): a box handed to the TMA unit
+        // is waited for (read out of shared memory) there, as late as possible.
+        auto stage_free = [&]() {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+        };
+        auto reduce = [&](const CUtensorMap* map, float* gbase, int heads, int head, int row0, int valid, int col) {
+            if (wq * 32 + 32 <= valid) {
+                fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_3d(map, warp_stage, col, head, row0 + wq * 32);
+                    bulk_commit_group();
+                }
+            } else {
+                __syncwarp();
+                const int sub = lane >> 3, chunk = lane & 7;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int rr = 4 * j + sub;
+                    const int q = wq * 32 + rr;
+                    if (q < valid) {
+                        const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
+                        red_add_v4(gbase + ((int64_t)(row0 + q) * heads + head) * kD + col + 4 * chunk, x.x, x.y,
+                                   x.z, x.w);
+                    }
+                }
+                __syncwarp();
+            }
+        };
+        // dQ(it) = dS K of this key tile, rows = the step's query rows: read out of Y (which
+        // is then released for b(it+1)) and added, times scale, into the fp32 dQ.
         auto drain = [&](int it, const StepMeta& mt, int h) {
             mbar_wait(smem_u32(&bars->dq_full), it & 1, abort, a.status, 70);
             tc_fence_after();
-            const float sc = a.scale;
-            const bool whole = wq * 32 + 32 <= mt.m;
             uint32_t v[32];
-            auto stage = [&]() {  // this lane's 128-byte row segment, chunks swizzled by lane % 8
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(warp_stage + lane * 128 + ((c ^ (lane & 7)) << 4),
-                                 __float_as_uint(__uint_as_float(v[4 * c]) * sc),
-                                 __float_as_uint(__uint_as_float(v[4 * c + 1]) * sc),
-                                 __float_as_uint(__uint_as_float(v[4 * c + 2]) * sc),
-                                 __float_as_uint(__uint_as_float(v[4 * c + 3]) * sc));
-            };
-            auto reduce = [&](int k) {
-                const int col = hf * 64 + 32 * k;
-                if (whole) {
-                    fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_reduce_add_3d(&tmDQ, warp_stage, col, h, mt.row0 + wq * 32);
-                        bulk_commit_group();
-                        bulk_wait_group_read0();   // the box has been read: the rows may be rewritten
-                    }
-                    __syncwarp();
-                } else {
-                    __syncwarp();
-                    const int sub = lane >> 3, chunk = lane & 7;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int rr = 4 * j + sub;
-                        const int q = wq * 32 + rr;
-                        if (q < mt.m) {
-                            const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
-                            red_add_v4(a.dq_acc + ((int64_t)(mt.row0 + q) * a.hq + h) * kD + col + 4 * chunk, x.x,
-                                       x.y, x.z, x.w);
-                        }
-                    }
-                    __syncwarp();
-                }
-            };
             tmem_ld32(tY + lane_addr + hf * 64, v);
             tmem_wait_ld();
-            stage();
+            stage(v, a.scale);
             tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
-            reduce(0);
-            stage();
-            reduce(1);
+            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.m, hf * 64);
+            stage_free();
+            stage(v, a.scale);
+            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.m, hf * 64 + 32);
         };
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
@@ -1040,6 +1068,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                                             p[ch * 32 + t + 1] * (__uint_as_float(dpv[t + 1]) - d2.y));
                     }
                     const int chunk = ch * 4 + j;
+                    if (ch == 0 && j == 0) stage_free();   // the drain's last box has been read
                     st_shared_v4(ds_row + ((chunk ^ (r & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
                 }
             }
@@ -1050,28 +1079,23 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         drain(n_it - 1, prev, prev_h);
         // ---------------------------------------------------- dK, dV epilogue
+        // This item's share of dK and dV (its list segment) is added into the outputs.
         mbar_wait(smem_u32(&bars->acc_done), 0, abort, a.status, 74);
         tc_fence_after();
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
             const uint32_t src = which == 0 ? tDK : tDV;
-            float* out = which == 0 ? a.dk : a.dv;
-            const float mul = which == 0 ? a.scale : 1.f;
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t v[32];
-                const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(src + lane_addr + c0, v);
+                tmem_ld32(src + lane_addr + hf * 64 + ch * 32, v);
                 tmem_wait_ld();
-                if (r < kn) {
-                    float4* dst = reinterpret_cast<float4*>(out + ((int64_t)(k0 + r) * a.hkv + g) * kD + c0);
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        dst[t] = make_float4(__uint_as_float(v[4 * t]) * mul, __uint_as_float(v[4 * t + 1]) * mul,
-                                             __uint_as_float(v[4 * t + 2]) * mul, __uint_as_float(v[4 * t + 3]) * mul);
-                }
+                stage_free();
+                stage(v, which == 0 ? a.scale : 1.f);
+                reduce(which == 0 ? &tmDK : &tmDV, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kn, hf * 64 + ch * 32);
             }
         }
+        stage_free();   // every box read before the CTA's shared memory is released
     }
     tc_fence_before();
     __syncthreads();
@@ -1081,7 +1105,8 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }  // namespace
 
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream) {
+                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int n_items_per_group, int num_sms,
+                     cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
     static const bool fused = [] {
         const char* e = getenv("THD_BWD_SPLIT");
@@ -1091,18 +1116,23 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
     if (fused) {
         static std::atomic<uint64_t> fused_configured{0};
         if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, fused_configured)) return -1;
-        bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.T * a.hq, a.hq, a.T);
+        CUtensorMap mdq, mdk, mdv;
+        if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&mdk, a.dk, a.T, a.hkv, kD) ||
+            !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD))
+            return -1;
+        bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.dk, a.dv, a.T * a.hkv,
+                                                         a.T * a.hq, a.hq, a.T);
         if (cudaGetLastError() != cudaSuccess) return -1;
-        CUtensorMap mdq;
-        if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD)) return -1;
-        bwd_fused_kernel<<<kv_grid, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, a);
+        const unsigned items = (unsigned)((int64_t)n_items_per_group * a.hkv);
+        bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, a);
         return cudaGetLastError() == cudaSuccess ? 0 : -1;
     }
     static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};
     if (!ensure_dynamic_smem(dkdv_kernel, DkdvLayout::kBytes, dkdv_configured) ||
         !ensure_dynamic_smem(dq_kernel, DqLayout::kBytes, dq_configured))
         return -1;
-    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, nullptr, a.T * a.hq, a.hq, a.T);
+    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, nullptr, nullptr, nullptr, 0,
+                                                     a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
     dkdv_kernel<<<kv_grid, kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);
     if (cudaGetLastError() != cudaSuccess) return -1;

@@ -99,7 +99,9 @@ __device__ __forceinline__ int visible_prefix(int qpos, int nvalid, int kpos0, i
 template <int DQK, int DV, bool SHARED_ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKr, FwdArgs a) {
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKr,
+           const __grid_constant__ CUtensorMap tmQg, const __grid_constant__ CUtensorMap tmKg,
+           const __grid_constant__ CUtensorMap tmVg, FwdArgs a) {
     static_assert(!SHARED_ROPE || DQK == 192, "the shared rope key is the third 64-column box");
     using L = FwdLayout<DQK, DV>;
     constexpr int NK = L::NK, NV = L::NV;
@@ -151,47 +153,88 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t tmem = bars->tmem_base;
 
     if (warp == 0 || warp == 2) {
-        if (lane == 0) {
-            // ------------------------------------------------ TMA producers: warp 0 Q and K, warp 2 V
-            const bool is_k = warp == 0;
-            if (is_k) {
+        // ---------------------------------------------------- TMA producers: warp 0 Q and K, warp 2 V
+        // A rank-major tile (row0 / k0 >= 0) is a box of 128 consecutive rank-major rows,
+        // loaded by lane 0.  A position tile (row0 / k0 < 0; short-chunk documents) holds
+        // positions pos0 .. pos0+n-1, read in place from the rank-major buffer through
+        // rm_of_global: every lane gathers 4 rows per 64-column box (tile::gather4), rows
+        // past n repeat row n-1 (they are masked).
+        const bool is_k = warp == 0;
+        // this lane's 4 rows of a position tile (their indices are loaded one tile ahead,
+        // so that the load latency overlaps the wait for a free stage)
+        auto gather_index = [&](int pos0, int n, int heads, int head, int (&rr)[4]) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1)) * heads + head;
+        };
+        auto gather_rows = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int nbox) {
+            for (int c = 0; c < nbox; ++c)
+                tma_gather4(map, dst + c * L::kBox + lane * 512, bar, c * 64, rr[0], rr[1], rr[2], rr[3]);
+        };
+        if (is_k) {
+            if (lane == 0) {
                 tma_prefetch_desc(&tmQ);
                 tma_prefetch_desc(&tmK);
                 if (SHARED_ROPE) tma_prefetch_desc(&tmKr);
-                const uint32_t qf = smem_u32(&bars->q_full);
-                mbar_arrive_expect_tx(qf, L::kQBytes);
-                for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
-            } else {
-                tma_prefetch_desc(&tmV);
             }
-            const int ns = is_k ? NK : NV;
-            int k0_next = nk > 0 ? __ldg(E) : 0;
-            for (int j = 0; j < nk; ++j) {
-                const int st = j % ns;
-                const int k0 = k0_next;
-                if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
-                // A stage is refilled once the MMA that read it has retired: K_{j-NK} is
-                // read by S_{j-NK} (signalled on s_full), V_{j-NV} by PV_{j-NV} (o_done).
-                // NK, NV <= kSBuf, so the next use of either barrier needs the tile
-                // being loaded here: the awaited phase is never ambiguous.
-                if (is_k) {
-                    if (j >= NK)
-                        mbar_wait(smem_u32(&bars->s_full[(j - NK) % kSBuf]), ((j - NK) / kSBuf) & 1, abort, a.status, 1);
-                    const uint32_t kf = smem_u32(&bars->k_full[st]);
-                    mbar_arrive_expect_tx(kf, L::kKBytes);
-                    for (int c = 0; c < DQK / 64; ++c) {
-                        if (SHARED_ROPE && c == 2)
-                            tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, k0);
-                        else
-                            tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, k0);
-                    }
-                } else {
-                    if (j >= NV)
-                        mbar_wait(smem_u32(&bars->o_done[(j - NV) % kSBuf]), ((j - NV) / kSBuf) & 1, abort, a.status, 9);
-                    const uint32_t vf = smem_u32(&bars->v_full[st]);
-                    mbar_arrive_expect_tx(vf, L::kVBytes);
-                    for (int c = 0; c < DV / 64; ++c)
-                        tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, k0);
+            const uint32_t qf = smem_u32(&bars->q_full);
+            if (lane == 0) mbar_arrive_expect_tx(qf, L::kQBytes);
+            __syncwarp();
+            if (row0 >= 0) {
+                if (lane == 0)
+                    for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
+            } else if (!SHARED_ROPE) {
+                int rq[4];
+                gather_index(qpos0, m, a.hq, h, rq);
+                gather_rows(&tmQg, sQ, qf, rq, DQK / 64);
+            }
+        } else if (lane == 0) {
+            tma_prefetch_desc(&tmV);
+        }
+        const int ns = is_k ? NK : NV;
+        int4 e_next = nk > 0 ? __ldg(reinterpret_cast<const int4*>(E)) : make_int4(0, 0, 0, 0);
+        int rr_next[4] = {0, 0, 0, 0};
+        if (!SHARED_ROPE && nk > 0 && e_next.x < 0) gather_index(e_next.z, e_next.y, a.hkv, g, rr_next);
+        for (int j = 0; j < nk; ++j) {
+            const int st = j % ns;
+            const int4 e = e_next;   // k0, nvalid, kpos0, -
+            int rr[4] = {rr_next[0], rr_next[1], rr_next[2], rr_next[3]};
+            if (j + 1 < nk) {
+                e_next = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
+                if (!SHARED_ROPE && e_next.x < 0) gather_index(e_next.z, e_next.y, a.hkv, g, rr_next);
+            }
+            // A stage is refilled once the MMA that read it has retired: K_{j-NK} is
+            // read by S_{j-NK} (signalled on s_full), V_{j-NV} by PV_{j-NV} (o_done).
+            // NK, NV <= kSBuf, so the next use of either barrier needs the tile
+            // being loaded here: the awaited phase is never ambiguous.
+            if (is_k) {
+                if (j >= NK)
+                    mbar_wait(smem_u32(&bars->s_full[(j - NK) % kSBuf]), ((j - NK) / kSBuf) & 1, abort, a.status, 1);
+                const uint32_t kf = smem_u32(&bars->k_full[st]);
+                if (lane == 0) mbar_arrive_expect_tx(kf, L::kKBytes);
+                __syncwarp();
+                if (e.x >= 0) {
+                    if (lane == 0)
+                        for (int c = 0; c < DQK / 64; ++c) {
+                            if (SHARED_ROPE && c == 2)
+                                tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, e.x);
+                            else
+                                tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, e.x);
+                        }
+                } else if (!SHARED_ROPE) {
+                    gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, DQK / 64);
+                }
+            } else {
+                if (j >= NV)
+                    mbar_wait(smem_u32(&bars->o_done[(j - NV) % kSBuf]), ((j - NV) / kSBuf) & 1, abort, a.status, 9);
+                const uint32_t vf = smem_u32(&bars->v_full[st]);
+                if (lane == 0) mbar_arrive_expect_tx(vf, L::kVBytes);
+                __syncwarp();
+                if (e.x >= 0) {
+                    if (lane == 0)
+                        for (int c = 0; c < DV / 64; ++c)
+                            tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, e.x);
+                } else if (!SHARED_ROPE) {
+                    gather_rows(&tmVg, sV + st * L::kVBytes, vf, rr, DV / 64);
                 }
             }
         }
@@ -369,7 +412,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         named_bar_sync(2 + wq, 64);
         const float l_tot = l_run + xch[(hf ^ 1) * 128 + row];
         const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-        __nv_bfloat16* orow = a.o + ((size_t)(row0 + row) * a.hq + h) * DV + hf * (DV / 2);
+        // rank-major row of this query row (position tiles: through rm_of_global)
+        const int orow_idx = row0 >= 0 ? row0 + row : (row < m ? __ldg(a.rm_of_global + qpos0 + row) : 0);
+        __nv_bfloat16* orow = a.o + ((size_t)orow_idx * a.hq + h) * DV + hf * (DV / 2);
 #pragma unroll
         for (int c = 0; c < DV / 64; ++c) {
             uint32_t o[32];
@@ -386,7 +431,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
         }
         if (row < m && hf == 0)
-            a.lse[(size_t)h * a.T + row0 + row] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+            a.lse[(size_t)h * a.T + orow_idx] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
     }
     tc_fence_before();
     __syncthreads();
@@ -395,27 +440,31 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 template <int DQK, int DV, bool SHARED_ROPE>
-int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr, const FwdArgs& a,
-           int n_items, cudaStream_t stream) {
+int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr,
+           const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a, int n_items,
+           cudaStream_t stream) {
     using L = FwdLayout<DQK, DV>;
     static std::atomic<uint64_t> configured{0};
     if (!ensure_dynamic_smem(fwd_kernel<DQK, DV, SHARED_ROPE>, L::kDynSmem, configured)) return -1;
-    fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, a);
+    fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, qg, kg, vg, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 }  // namespace
 
 int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const FwdArgs& a, int n_items, cudaStream_t stream) {
-    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, a, n_items, stream);
-    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, a, n_items, stream);
+                     const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a,
+                     int n_items, cudaStream_t stream) {
+    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, qg, kg, vg, a, n_items, stream);
+    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, qg, kg, vg, a, n_items, stream);
     return -2;
 }
 
+// The compact-key form walks rank-major tiles only (the tables it is given have no
+// position tiles), so its row maps are never read.
 int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
                          const CUtensorMap& v, const FwdArgs& a, int n_items, cudaStream_t stream) {
-    return launch<192, 128, true>(q, k_nope, v, k_rope, a, n_items, stream);
+    return launch<192, 128, true>(q, k_nope, v, k_rope, q, k_nope, v, a, n_items, stream);
 }
 
 }  // namespace thd

@@ -87,6 +87,8 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     a.kt_off = plan->d_kt_off;
     a.kt_list = plan->d_kt_list;
     a.kt_lpt = plan->d_kt_lpt;
+    a.kt_seg = plan->d_kt_seg;
+    a.n_kseg = (int32_t)(plan->kt_seg.size() - 1);
     a.o = static_cast<const __nv_bfloat16*>(o_rm);
     a.dout = static_cast<const __nv_bfloat16*>(do_rm);
     a.lse = lse_rm;
@@ -101,7 +103,7 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = plan->d_status;
     if (plan->n_qtiles() == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)plan->n_qtiles(), sm_count(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)plan->n_qtiles(), plan->kt_seg.back(), sm_count(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

@@ -27,6 +27,9 @@ inline bool ensure_dynamic_smem(Kernel* fn, int bytes, std::atomic<uint64_t>& do
 // 128-row boxes and 128-byte swizzle (the layout the tcgen05 descriptors expect).
 // False when the driver's encoder is unavailable or rejects the map.
 bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
+// [rows, dim] bf16 tensor (a [T, heads, dim] tensor seen as T * heads rows) viewed as a
+// 2-D TMA map with 64-column x 1-row boxes and 128-byte swizzle, for tile::gather4 loads.
+bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int dim);
 // [rows, heads, dim] fp32 tensor viewed as a 3-D TMA map with 32-column x 1-head x 32-row
 // boxes (128-byte rows) and 128-byte swizzle: the target of tiled reductions.
 bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
@@ -42,6 +45,7 @@ struct FwdArgs {
     const int32_t* qtiles;
     const int32_t* entries;
     const int32_t* lpt;
+    const int32_t* rm_of_global;  // rows of position tiles (row0 / k0 < 0)
     __nv_bfloat16* o;
     float* lse;
     int32_t hq, hkv;
@@ -49,8 +53,10 @@ struct FwdArgs {
     float scale_log2;  // scale * log2(e)
     int* status;       // device word: nonzero once a bounded wait gave up
 };
+// qg, kg, vg: the same tensors as 2-D row maps (make_map_bf16_rows), read by position tiles.
 int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const FwdArgs& a, int n_items, cudaStream_t stream);
+                     const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a,
+                     int n_items, cudaStream_t stream);
 // Multi-head latent attention with a shared rope key: Q [T, hq, 192], K_nope [T, hkv, 128],
 // K_rope [T, 1, 64] (one per token, every head), V [T, hkv, 128].
 int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
@@ -80,6 +86,8 @@ struct BwdArgs {
     const int32_t* kt_off;
     const int32_t* kt_list;
     const int32_t* kt_lpt;
+    const int32_t* kt_seg;  // backward work items by list segment (THD_KSEG entries each)
+    int32_t n_kseg;
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;
     const float* lse;
@@ -93,8 +101,11 @@ struct BwdArgs {
     float scale_log2;
     int* status;
 };
+// n_tiles: key tiles; n_items_per_group: backward work items per key/value head
+// (kt_seg[n_kseg], the list segments of every key tile).
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int num_sms, cudaStream_t stream);
+                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int n_items_per_group, int num_sms,
+                     cudaStream_t stream);
 
 // ---- rotary position embedding (half-split), per-document positions ---------------
 int launch_rope(__nv_bfloat16* x, const int32_t* pos, int64_t T, int heads, int dim, int rot_dim, double base,

@@ -214,6 +214,62 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         std::stable_sort(p->kt_lpt.begin(), p->kt_lpt.end(), [&](int32_t a, int32_t b) {
             return p->kt_off[a + 1] - p->kt_off[a] > p->kt_off[b + 1] - p->kt_off[b];
         });
+        // Backward work items: segment j of every key tile whose list reaches it.  kt_lpt
+        // is by descending list length, so those key tiles are its first n_j entries.
+        const int64_t max_len = n_tiles ? (int64_t)p->kt_off[p->kt_lpt[0] + 1] - p->kt_off[p->kt_lpt[0]] : 0;
+        const int64_t n_seg = ceil_div(max_len, THD_KSEG);
+        p->kt_seg.assign(n_seg + 1, 0);
+        int64_t reach = n_tiles;  // key tiles whose list is longer than j * THD_KSEG
+        for (int64_t j = 0; j < n_seg; ++j) {
+            while (reach > 0 && (int64_t)p->kt_off[p->kt_lpt[reach - 1] + 1] - p->kt_off[p->kt_lpt[reach - 1]] <=
+                                    j * THD_KSEG)
+                --reach;
+            p->kt_seg[j + 1] = (int32_t)(p->kt_seg[j] + reach);
+        }
+
+        // ---- forward tables -------------------------------------------------
+        // A document whose chunks are shorter than a tile (c < BM) puts two or more
+        // chunks, far apart in position, into every rank-major tile, so that most of
+        // each tile pair is masked.  The forward tiles such a document in position
+        // order instead: query tile u and key tile v are positions s + u*BM .. and
+        // s + v*BM .. (read in place from the rank-major buffers through rm_of_global),
+        // key tiles 0 .. u listed for query tile u, the last one the diagonal.  Rank-major
+        // records are marked by row0 / k0 >= 0; position records carry -1 there.
+        p->fqtiles.clear();
+        p->fentries.clear();
+        for (int64_t t = 0; t < n_tiles; ++t) {
+            const int32_t* q = &p->qtiles[(size_t)t * THD_QTILE_FIELDS];
+            if (lay.chunk(q[1]) < BM) continue;
+            const int32_t off = (int32_t)(p->fentries.size() / THD_ENTRY_FIELDS);
+            p->fqtiles.insert(p->fqtiles.end(), q, q + THD_QTILE_FIELDS);
+            p->fqtiles[p->fqtiles.size() - THD_QTILE_FIELDS + 9] = off;
+            p->fentries.insert(p->fentries.end(), p->entries.begin() + (size_t)q[9] * THD_ENTRY_FIELDS,
+                               p->entries.begin() + (size_t)(q[9] + q[8]) * THD_ENTRY_FIELDS);
+        }
+        for (int d = 0; d < n_docs; ++d) {
+            if (lay.chunk(d) >= BM) continue;
+            const int64_t n = ceil_div(L[d], BM);
+            for (int64_t u = 0; u < n; ++u) {
+                const int64_t p0 = s[d] + u * BM, m = std::min<int64_t>(BM, L[d] - u * BM), qmax = p0 + m - 1;
+                const int32_t rec[THD_QTILE_FIELDS] = {-1, d, -1, (int32_t)m, (int32_t)p0, (int32_t)m, 0, (int32_t)qmax,
+                                                       (int32_t)(u + 1),
+                                                       (int32_t)(p->fentries.size() / THD_ENTRY_FIELDS),
+                                                       (int32_t)s[d], (int32_t)(s[d] + L[d])};
+                p->fqtiles.insert(p->fqtiles.end(), rec, rec + THD_QTILE_FIELDS);
+                for (int64_t v = 0; v <= u; ++v) {
+                    const int64_t kp0 = s[d] + v * BM, nv = std::min<int64_t>(BM, qmax - kp0 + 1);
+                    const int32_t cls = kp0 + nv - 1 <= p0 ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
+                    const int32_t e[THD_ENTRY_FIELDS] = {-1, (int32_t)nv, (int32_t)kp0, (int32_t)nv, 0, cls, -1, -1};
+                    p->fentries.insert(p->fentries.end(), e, e + THD_ENTRY_FIELDS);
+                }
+            }
+        }
+        const int64_t nf = (int64_t)p->fqtiles.size() / THD_QTILE_FIELDS;
+        p->flpt.resize(nf);
+        for (int64_t t = 0; t < nf; ++t) p->flpt[t] = (int32_t)t;
+        std::stable_sort(p->flpt.begin(), p->flpt.end(), [&](int32_t a, int32_t b) {
+            return p->fqtiles[(size_t)a * THD_QTILE_FIELDS + 8] > p->fqtiles[(size_t)b * THD_QTILE_FIELDS + 8];
+        });
     } catch (const std::bad_alloc&) {
         return THD_ERR_ALLOC;
     }

@@ -17,7 +17,10 @@ struct thd_cp_plan_s {
     // host tables (see thd_cp_plan_export for the record layouts)
     std::vector<int32_t> q_idx, rm_of_global;
     std::vector<int32_t> qtiles, entries, lpt;
-    std::vector<int32_t> kt_off, kt_list, kt_lpt;
+    std::vector<int32_t> kt_off, kt_list, kt_lpt, kt_seg;
+    // forward tables: rank-major tiles of documents whose chunks span a tile or more,
+    // position-ordered tiles of documents with shorter chunks
+    std::vector<int32_t> fqtiles, fentries, flpt;
 
     // Device side, valid after thd_cp_plan_upload.  Every table lives in one
     // stream-ordered allocation (d_buf, grown only when a layout needs more), and
@@ -33,11 +36,14 @@ struct thd_cp_plan_s {
     int next_stage = 0;
     int32_t *d_q_idx = nullptr, *d_rm_of_global = nullptr;
     int32_t *d_qtiles = nullptr, *d_entries = nullptr, *d_lpt = nullptr;
-    int32_t *d_kt_off = nullptr, *d_kt_list = nullptr, *d_kt_lpt = nullptr;
+    int32_t *d_kt_off = nullptr, *d_kt_list = nullptr, *d_kt_lpt = nullptr, *d_kt_seg = nullptr;
+    int32_t *d_fqtiles = nullptr, *d_fentries = nullptr, *d_flpt = nullptr;
     int32_t* d_status = nullptr;  // set by kernels whose bounded waits gave up
 
     int64_t n_qtiles() const { return (int64_t)qtiles.size() / THD_QTILE_FIELDS; }
     int64_t n_entries() const { return (int64_t)entries.size() / THD_ENTRY_FIELDS; }
+    int64_t n_fqtiles() const { return (int64_t)fqtiles.size() / THD_QTILE_FIELDS; }
+    int64_t n_fentries() const { return (int64_t)fentries.size() / THD_ENTRY_FIELDS; }
 };
 
 // THD_OK when the plan's tables are on the device, that device is current and no

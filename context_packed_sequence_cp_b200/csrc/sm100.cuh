@@ -100,6 +100,18 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint32_t sme
         : "memory");
 }
 
+// Four rows of a 2-D tensor map whose box is one row high (box width x 1), at arbitrary
+// row coordinates, land as four consecutive box rows at smem_dst (tile::gather4, no
+// multicast); completion counted in bytes on the mbarrier.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint32_t smem_dst, uint32_t bar, int32_t col,
+                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // 3-D tiled reduction (add) of a shared-memory box into global memory, tracked as a
 // bulk async-group of the issuing thread.  The box's innermost coordinate times the
 // element size is a multiple of 16 bytes; coordinates are non-negative.

@@ -68,6 +68,9 @@ extern "C" {
 #define THD_ENTRY_FIELDS 8
 #define THD_CLS_PARTIAL  1
 #define THD_CLS_UNMASKED 2
+/* Query tiles per backward work item: a key tile's list is walked in segments of this
+ * many entries (part of the plan's contract, see kt_seg). */
+#define THD_KSEG 32
 
 typedef struct thd_cp_plan_s* thd_cp_plan_t;   /* opaque, library-owned */
 
@@ -79,6 +82,9 @@ typedef struct thd_cp_plan_info_s {
     int64_t n_qtiles;   /* 128-row tiles (query tiles == key tiles)              */
     int64_t n_entries;  /* listed (query tile, key tile) pairs                   */
     int64_t causal_pairs; /* sum over documents of L (L + 1) / 2                 */
+    int64_t n_kseg;     /* segments of the longest key-tile list (THD_KSEG entries each) */
+    int64_t n_fqtiles;  /* query tiles of the forward tables (thd_cp_plan_export_fwd)   */
+    int64_t n_fentries; /* entries of the forward tables                                */
 } thd_cp_plan_info_t;
 
 /*
@@ -176,10 +182,36 @@ int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out);
  *   kt_list      int32[n_entries*2] (qtile, entry) per key tile, by descending
  *                qpos_max of the query tile (ties by qtile index)
  *   kt_lpt       int32[n_qtiles]   key tiles by descending list length
+ *   kt_seg       int32[n_kseg+1]   backward work items by segment: a key tile's list
+ *                is cut into segments of THD_KSEG entries; kt_seg[j+1] - kt_seg[j] is the
+ *                number of key tiles whose list reaches segment j (the first ones of
+ *                kt_lpt), kt_seg[0] = 0.  Lists being prefixes of one order per
+ *                document, segment j of every key tile of a document walks the same
+ *                query tiles.
  */
 int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global,
                        int32_t* qtiles, int32_t* entries, int32_t* lpt,
-                       int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt);
+                       int32_t* kt_off, int32_t* kt_list, int32_t* kt_lpt, int32_t* kt_seg);
+
+/*
+ * thd_cp_plan_export_fwd -- copy the forward tables into caller-allocated host arrays
+ * (NULL skips a table).  Documents whose chunks are shorter than a tile
+ * (L / (2 cp) < THD_BM) put two or more chunks, far apart in position, into every
+ * rank-major tile, so that most of each tile pair is masked ([WHAT] one fused call
+ * over all documents: short documents must not waste it).  The forward tiles them in
+ * position order, reading the rank-major buffers in place through rm_of_global:
+ *   fqtiles   int32[n_fqtiles * 12], qtile layout.  First the rank-major query tiles
+ *             of the other documents (as in qtiles, entry_off into fentries), then, per
+ *             short-chunk document d (ascending) and u = 0 .. ceil(L/128)-1, a position
+ *             tile: r = -1, d, row0 = -1, m = min(128, L - 128u), qpos0 = s_d + 128u,
+ *             qbrk = m, qjump = 0, qpos_max, nk = u + 1, entry_off, doc_start, doc_end.
+ *   fentries  int32[n_fentries * 8], entry layout.  For a position tile, its key tiles
+ *             v = 0 .. u: k0 = -1, nvalid (128, or m for v = u), kpos0 = s_d + 128v,
+ *             kbrk = nvalid, kjump = 0, cls (UNMASKED below the diagonal), ktile = -1,
+ *             key_rank = -1.
+ *   flpt      int32[n_fqtiles]  forward query tiles by descending nk (ties by index).
+ */
+int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt);
 
 /*
  * thd_cp_plan_upload -- copy the tables to the current device once and keep them

@@ -32,7 +32,9 @@ Record layouts (int32):
   kt_off[n_tiles+1] / kt_list[n_entries][2] = (qtile, entry), each key tile's list
   in descending order of the q-tile's qpos_max (ties by q-tile index).
   lpt: q-tiles by descending nk (ties by index); kt_lpt: key tiles by descending
-  number of listed q-tiles (ties by index).
+  number of listed q-tiles (ties by index); kt_seg[j+1] - kt_seg[j]: the number of key
+  tiles whose list has more than j*KSEG entries (segments of KSEG = 32 entries are
+  the backward's work items), kt_seg[0] = 0.
 
 Everything is derived from the explicit partition (``partition.partition``) by
 enumerating every (query row, key row) pair of a tile; nothing uses the closed-form
@@ -46,6 +48,7 @@ from .partition import partition, doc_of_token, validate
 
 BM = 128
 BN = 128
+KSEG = 32           # key-tile list entries per backward work item
 PARTIAL = 1
 UNMASKED = 2
 QT_FIELDS = 12
@@ -133,10 +136,60 @@ def tile_plan(cu_seqlens, cp: int) -> dict:
     kt_list = np.array([p for x in lists for p in sorted(x, key=lambda pr: (-int(qtiles[pr[0], 7]), pr[0]))],
                        dtype=np.int32).reshape(-1, 2)
     kt_lpt = np.array(sorted(range(n_tiles), key=lambda t: (-len(lists[t]), t)), dtype=np.int32)
+    # backward work items: segment j (entries j*KSEG .. j*KSEG+KSEG-1) of every key tile
+    # whose list is longer than j*KSEG; kt_seg holds their running count per segment
+    n_seg = -(-max((len(x) for x in lists), default=0) // KSEG)
+    kt_seg = np.zeros(n_seg + 1, dtype=np.int32)
+    for j in range(n_seg):
+        kt_seg[j + 1] = kt_seg[j] + sum(1 for x in lists if len(x) > j * KSEG)
 
+    fqtiles, fentries, flpt = _forward_tables(cu, cp, qtiles, entries)
     return dict(T=int(cu[-1]), cp=int(cp), Tl=int(cu[-1]) // cp, n_docs=n_docs,
                 q_idx=q_idx, rm_of_global=rm_of_global, qtiles=qtiles, entries=entries,
-                lpt=lpt, kt_off=kt_off, kt_list=kt_list, kt_lpt=kt_lpt)
+                lpt=lpt, kt_off=kt_off, kt_list=kt_list, kt_lpt=kt_lpt, kt_seg=kt_seg,
+                fqtiles=fqtiles, fentries=fentries, flpt=flpt)
+
+
+def _forward_tables(cu, cp, qtiles, entries):
+    """The forward's tiles.  A document whose chunks are shorter than a tile
+    (L / (2 cp) < 128) is tiled in position order: query tile u holds positions
+    s + 128u .. (up to 128), and every key tile v (positions s + 128v ..) holding a key
+    that some of its queries can see is listed, found by enumerating the (query, key)
+    pairs; row0 / k0 / r / ktile / key_rank are -1 for these records (the rows are
+    found through rm_of_global).  Other documents keep their rank-major tiles, in the
+    order of the main table, first."""
+    n_docs = cu.size - 1
+    short = {d for d in range(n_docs) if (int(cu[d + 1]) - int(cu[d])) // (2 * cp) < BM}
+    fq, fe = [], []
+    for t in range(qtiles.shape[0]):
+        if int(qtiles[t, 1]) in short:
+            continue
+        rec = qtiles[t].copy()
+        e0, nk = int(rec[9]), int(rec[8])
+        rec[9] = len(fe)
+        fq.append(rec)
+        fe.extend(entries[e0:e0 + nk].tolist())
+    for d in sorted(short):
+        s, e = int(cu[d]), int(cu[d + 1])
+        for p0 in range(s, e, BM):
+            qpos = np.arange(p0, min(p0 + BM, e))
+            first = len(fe)
+            for k0 in range(s, e, BN):
+                kpos = np.arange(k0, min(k0 + BN, e))
+                vis = kpos[None, :] <= qpos[:, None]
+                seen = vis.any(axis=0)
+                nv = int(seen.sum())
+                if nv == 0:
+                    continue
+                assert seen[:nv].all(), "visible keys of a position tile form a prefix"
+                cls = UNMASKED if vis[:, :nv].all() else PARTIAL
+                fe.append([-1, nv, int(kpos[0]), nv, 0, cls, -1, -1])
+            fq.append(np.array([-1, d, -1, qpos.size, int(qpos[0]), qpos.size, 0, int(qpos[-1]),
+                                len(fe) - first, first, s, e], dtype=np.int32))
+    fqtiles = np.array(fq, dtype=np.int32).reshape(-1, QT_FIELDS)
+    fentries = np.array(fe, dtype=np.int32).reshape(-1, EN_FIELDS)
+    flpt = np.array(sorted(range(fqtiles.shape[0]), key=lambda t: (-int(fqtiles[t, 8]), t)), dtype=np.int32)
+    return fqtiles, fentries, flpt
 
 
 def decode_run(pos0: int, brk: int, jump: int, n: int) -> np.ndarray:

@@ -122,3 +122,21 @@ def test_fwd_rejects_unsupported_dims():
     with pytest.raises(thd.ThdError) as e:
         thd.thd_cp_attn_fwd(plan, x, x, x)
     assert e.value.kind == "UNSUPPORTED"
+
+
+@pytest.mark.parametrize("cp", [2, 4])
+def test_fwd_bf16_position_tiles_around_the_chunk_threshold(cp):
+    """Documents whose chunks are shorter than a tile are tiled in position order (their
+    rows gathered through rm_of_global), the others rank-major: chunk sizes 1, 17, 64,
+    127 (position tiles) and 128, 129, 300 (rank-major) in one packed sequence, GQA 8/2,
+    every output compared."""
+    chunks = [1, 17, 64, 127, 128, 129, 300, 3]
+    lens = [2 * cp * c for c in chunks]
+    cu = syn.cu_seqlens_of(lens)
+    q, k, v = syn.make_tensors(int(cu[-1]), 8, 2, 128, 128, torch.bfloat16, seed=40 + cp)
+    o, lse, plan, _ = run_forward(cu, cp, q, k, v)
+    fwd = plan.export_fwd()
+    assert (fwd["fqtiles"][:, 2] < 0).any() and (fwd["fqtiles"][:, 2] >= 0).any()
+    want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
+    assert_bf16_close(o, want_o, "O")
+    assert np.abs(lse - want_l).max() <= LSE_MAX

@@ -118,6 +118,45 @@ def test_tiles_cover_every_visible_pair_once(seed):
         assert total == P.causal_pairs_total(cu)
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_forward_tables_cover_every_visible_pair_once(seed):
+    """The forward tables (rank-major tiles, position tiles for short-chunk documents)
+    list every visible (query, key) pair exactly once, every query row of the packed
+    sequence in exactly one query tile, and classes that match the pairs."""
+    for cp, cu in _layouts(12, cps=(1, 2, 4, 8), T_max=1500, seed=300 + seed):
+        plan = TT.tile_plan(cu, cp)
+        doc = P.doc_of_token(cu)
+        seen_q = np.zeros(int(cu[-1]), dtype=np.int64)
+        total = 0
+        for q in plan["fqtiles"]:
+            r, d, row0, m, qpos0, qbrk, qjump, qmax, nk, e0, ds, de = (int(x) for x in q)
+            qpos = TT.decode_run(qpos0, qbrk, qjump, m)
+            if row0 >= 0:
+                assert np.array_equal(plan["q_idx"][row0:row0 + m], qpos)
+            else:   # position tile of a short-chunk document
+                assert (de - ds) // (2 * cp) < TT.BM and r == -1
+                assert np.array_equal(qpos, np.arange(qpos0, qpos0 + m))
+            assert np.all(doc[qpos] == d) and qmax == qpos[-1]
+            seen_q[qpos] += 1
+            for en in plan["fentries"][e0:e0 + nk]:
+                kpos = TT.decode_run(int(en[2]), int(en[3]), int(en[4]), int(en[1]))
+                if en[0] >= 0:
+                    assert np.array_equal(plan["q_idx"][en[0]:en[0] + en[1]], kpos)
+                assert np.all(doc[kpos] == d)
+                vis = kpos[None, :] <= qpos[:, None]
+                cnt = int(vis.sum())
+                assert cnt > 0 and vis.any(axis=0).all()
+                assert (en[5] == TT.UNMASKED) == bool(vis.all())
+                total += cnt
+        assert np.all(seen_q == 1)
+        assert total == P.causal_pairs_total(cu)
+        order = plan["flpt"]
+        assert sorted(order.tolist()) == list(range(plan["fqtiles"].shape[0]))
+        nk = plan["fqtiles"][:, 8]
+        for a, b in zip(order[:-1], order[1:]):
+            assert nk[a] > nk[b] or (nk[a] == nk[b] and a < b)
+
+
 def test_tiles_pairwise_bruteforce_tiny():
     """Every visible (query, key) pair of the packed sequence lies in exactly one
     listed entry of its query's tile; checked pair by pair."""

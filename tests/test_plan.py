@@ -9,7 +9,8 @@ from context_packed_sequence_cp_b200 import synthetic as syn
 from oracle import partition as P
 from oracle import tiles as TT
 
-KEYS = ("q_idx", "rm_of_global", "qtiles", "entries", "lpt", "kt_off", "kt_list", "kt_lpt")
+KEYS = ("q_idx", "rm_of_global", "qtiles", "entries", "lpt", "kt_off", "kt_list", "kt_lpt", "kt_seg")
+FWD_KEYS = ("fqtiles", "fentries", "flpt")
 
 
 def _compare(cu, cp):
@@ -20,6 +21,9 @@ def _compare(cu, cp):
     assert got.causal_pairs == P.causal_pairs_total(cu)
     for k in KEYS:
         assert np.array_equal(ex[k], want[k].reshape(ex[k].shape)), k
+    fx = got.export_fwd()
+    for k in FWD_KEYS:
+        assert np.array_equal(fx[k], want[k].reshape(fx[k].shape)), k
     got.close()
 
 
@@ -106,6 +110,9 @@ def test_plan_update_equals_a_fresh_plan():
         for k in KEYS:
             assert np.array_equal(ex[k], ref[k]), k
             assert np.array_equal(ex[k], want[k].reshape(ex[k].shape)), k
+        fx = plan.export_fwd()
+        for k in FWD_KEYS:
+            assert np.array_equal(fx[k], want[k].reshape(fx[k].shape)), k
         fresh.close()
     before = plan.export()
     with pytest.raises(ThdError) as e:
