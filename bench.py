@@ -564,7 +564,7 @@ def run_native(args):
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, cu, args.seed),
-        "roofline": {"kernel": "bwd (thd_cp_attn_bwd: prep + key-major dK/dV + query-major dQ tcgen05 kernels)", "bound": "tensor",
+        "roofline": {"kernel": "bwd (thd_cp_attn_bwd: prep + fused key-major dK/dV/dQ tcgen05 kernel)", "bound": "tensor",
                      "achieved": bwd_tf, "peak": sustained, "unit": "TFLOP/s", "frac": bwd_tf / sustained,
                      "traffic": traffic, "peak_source": f"bf16_tflops_sustained ({peak_src})",
                      "flops_per_launch": bwd_fl},

@@ -30,7 +30,7 @@ SIGNATURES = {
     "thd_cp_plan": (ctypes.c_int, [_PI32, _I32, _I32, ctypes.POINTER(_P)]),
     "thd_cp_plan_info": (ctypes.c_int, [_P, _P]),
     "thd_cp_plan_export": (ctypes.c_int, [_P, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32]),
-    "thd_cp_plan_export_fwd": (ctypes.c_int, [_P, _PI32, _PI32, _PI32]),
+    "thd_cp_plan_export_fwd": (ctypes.c_int, [_P, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32, _PI32]),
     "thd_cp_plan_upload": (ctypes.c_int, [_P, _P]),
     "thd_cp_plan_update": (ctypes.c_int, [_P, _PI32, _I32, _I32, _P]),
     "thd_cp_plan_destroy": (None, [_P]),
@@ -58,7 +58,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("cp", ctypes.c_int32), ("n_docs", ctypes.c_int32),
                 ("Tl", ctypes.c_int64), ("n_qtiles", ctypes.c_int64), ("n_entries", ctypes.c_int64),
                 ("causal_pairs", ctypes.c_int64), ("n_kseg", ctypes.c_int64), ("n_fqtiles", ctypes.c_int64),
-                ("n_fentries", ctypes.c_int64)]
+                ("n_fentries", ctypes.c_int64), ("n_fkseg", ctypes.c_int64)]
 
 
 class ThdError(RuntimeError):

@@ -124,10 +124,14 @@ class Plan:
 
     def export_fwd(self) -> dict:
         """The forward tables (thd_cp_plan_export_fwd)."""
-        out = dict(fqtiles=np.empty((self.n_fqtiles, QT_FIELDS), np.int32),
-                   fentries=np.empty((self.n_fentries, EN_FIELDS), np.int32), flpt=np.empty(self.n_fqtiles, np.int32))
+        nf, ne = self.n_fqtiles, self.n_fentries
+        out = dict(fqtiles=np.empty((nf, QT_FIELDS), np.int32), fentries=np.empty((ne, EN_FIELDS), np.int32),
+                   flpt=np.empty(nf, np.int32), fkt_off=np.empty(nf + 1, np.int32),
+                   fkt_list=np.empty((ne, 2), np.int32), fkt_lpt=np.empty(nf, np.int32),
+                   fkt_seg=np.empty(self.n_fkseg + 1, np.int32))
         check("thd_cp_plan_export_fwd", lib().thd_cp_plan_export_fwd(
-            self._h, _i32p(out["fqtiles"]), _i32p(out["fentries"]), _i32p(out["flpt"])))
+            self._h, *(_i32p(out[k]) for k in ("fqtiles", "fentries", "flpt", "fkt_off", "fkt_list", "fkt_lpt",
+                                                "fkt_seg"))))
         return out
 
     def upload(self, stream=None) -> "Plan":
@@ -172,6 +176,7 @@ class Plan:
         self.causal_pairs = int(info.causal_pairs)
         self.n_kseg = int(info.n_kseg)
         self.n_fqtiles, self.n_fentries = int(info.n_fqtiles), int(info.n_fentries)
+        self.n_fkseg = int(info.n_fkseg)
 
     def device_status(self, reset: bool = True) -> int:
         v = ctypes.c_int32()

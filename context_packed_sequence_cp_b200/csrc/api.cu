@@ -59,6 +59,7 @@ void free_device(thd_plan* p) {
     p->d_q_idx = p->d_rm_of_global = p->d_qtiles = p->d_entries = p->d_lpt = nullptr;
     p->d_kt_off = p->d_kt_list = p->d_kt_lpt = p->d_kt_seg = p->d_status = nullptr;
     p->d_fqtiles = p->d_fentries = p->d_flpt = nullptr;
+    p->d_fkt_off = p->d_fkt_list = p->d_fkt_lpt = p->d_fkt_seg = nullptr;
     p->uploaded = false;
 }
 
@@ -71,13 +72,15 @@ size_t round_up(size_t n) { return (n + kAlign - 1) & ~(kAlign - 1); }
 // tables outgrow it; the status word at its start survives a re-plan.  Work on `s`
 // enqueued earlier reads the previous tables before the copy overwrites them.
 int copy_tables(thd_plan* p, cudaStream_t s, bool first) {
-    constexpr int kTables = 12;
-    const std::vector<int32_t>* src[kTables] = {&p->q_idx,  &p->rm_of_global, &p->qtiles, &p->entries,
-                                                &p->lpt,    &p->kt_off,       &p->kt_list, &p->kt_lpt,
-                                                &p->kt_seg, &p->fqtiles,      &p->fentries, &p->flpt};
-    int32_t** dst[kTables] = {&p->d_q_idx,  &p->d_rm_of_global, &p->d_qtiles,  &p->d_entries,
-                              &p->d_lpt,    &p->d_kt_off,       &p->d_kt_list, &p->d_kt_lpt,
-                              &p->d_kt_seg, &p->d_fqtiles,      &p->d_fentries, &p->d_flpt};
+    constexpr int kTables = 16;
+    const std::vector<int32_t>* src[kTables] = {&p->q_idx,    &p->rm_of_global, &p->qtiles,   &p->entries,
+                                                &p->lpt,      &p->kt_off,       &p->kt_list,  &p->kt_lpt,
+                                                &p->kt_seg,   &p->fqtiles,      &p->fentries, &p->flpt,
+                                                &p->fkt_off,  &p->fkt_list,     &p->fkt_lpt,  &p->fkt_seg};
+    int32_t** dst[kTables] = {&p->d_q_idx,   &p->d_rm_of_global, &p->d_qtiles,   &p->d_entries,
+                              &p->d_lpt,     &p->d_kt_off,       &p->d_kt_list,  &p->d_kt_lpt,
+                              &p->d_kt_seg,  &p->d_fqtiles,      &p->d_fentries, &p->d_flpt,
+                              &p->d_fkt_off, &p->d_fkt_list,     &p->d_fkt_lpt,  &p->d_fkt_seg};
     size_t off[kTables];
     size_t total = kAlign;  // the status word (16 bytes) sits in the first 256
     for (int i = 0; i < kTables; ++i) {
@@ -216,6 +219,7 @@ int thd_cp_plan_info(thd_cp_plan_t plan, thd_cp_plan_info_t* out) {
     out->n_kseg = plan->kt_seg.empty() ? 0 : (int64_t)plan->kt_seg.size() - 1;
     out->n_fqtiles = plan->n_fqtiles();
     out->n_fentries = plan->n_fentries();
+    out->n_fkseg = plan->fkt_seg.empty() ? 0 : (int64_t)plan->fkt_seg.size() - 1;
     return THD_OK;
 }
 
@@ -238,7 +242,8 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
     return THD_OK;
 }
 
-int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt) {
+int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt,
+                           int32_t* fkt_off, int32_t* fkt_list, int32_t* fkt_lpt, int32_t* fkt_seg) {
     if (!plan) return THD_ERR_INVALID_ARG;
     auto cp = [](int32_t* dst, const std::vector<int32_t>& v) {
         if (dst && !v.empty()) std::memcpy(dst, v.data(), v.size() * sizeof(int32_t));
@@ -246,6 +251,10 @@ int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentri
     cp(fqtiles, plan->fqtiles);
     cp(fentries, plan->fentries);
     cp(flpt, plan->flpt);
+    cp(fkt_off, plan->fkt_off);
+    cp(fkt_list, plan->fkt_list);
+    cp(fkt_lpt, plan->fkt_lpt);
+    cp(fkt_seg, plan->fkt_seg);
     return THD_OK;
 }
 
@@ -294,6 +303,10 @@ int thd_cp_plan_update(thd_cp_plan_t plan, const int32_t* cu_seqlens, int32_t n_
     plan->fqtiles.swap(fresh.fqtiles);
     plan->fentries.swap(fresh.fentries);
     plan->flpt.swap(fresh.flpt);
+    plan->fkt_off.swap(fresh.fkt_off);
+    plan->fkt_list.swap(fresh.fkt_list);
+    plan->fkt_lpt.swap(fresh.fkt_lpt);
+    plan->fkt_seg.swap(fresh.fkt_seg);
     if (!plan->uploaded) return THD_OK;
     // On a failed copy the device tables no longer match the host tables: the plan
     // becomes not-uploaded, and a later thd_cp_plan_upload copies them afresh.
@@ -381,16 +394,19 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
     if (!aligned16(q_rm) || !aligned16(k_nope_rm) || !aligned16(k_rope_rm) || !aligned16(v_rm) || !aligned16(o_rm) ||
         !aligned16(lse_rm))
         return THD_ERR_MISALIGNED;
-    const int64_t items = plan->n_qtiles() * (int64_t)hq;
+    const int64_t items = plan->n_fqtiles() * (int64_t)hq;
     if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
-    CUtensorMap mq, mkn, mkr, mv;
+    CUtensorMap mq, mkn, mkr, mv, mqg, mkng, mkrg, mvg;
     if (!make_map_bf16(&mq, q_rm, plan->T, hq, d_nope + d_rope) || !make_map_bf16(&mkn, k_nope_rm, plan->T, hkv, d_nope) ||
-        !make_map_bf16(&mkr, k_rope_rm, plan->T, 1, d_rope) || !make_map_bf16(&mv, v_rm, plan->T, hkv, dv))
+        !make_map_bf16(&mkr, k_rope_rm, plan->T, 1, d_rope) || !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) ||
+        !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, d_nope + d_rope) ||
+        !make_map_bf16_rows(&mkng, k_nope_rm, plan->T * hkv, d_nope) ||
+        !make_map_bf16_rows(&mkrg, k_rope_rm, plan->T, d_rope) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
         return THD_ERR_CUDA;
-    thd::FwdArgs a;
-    a.qtiles = plan->d_qtiles;   // rank-major tiles only (position tiles are not built for the compact keys)
-    a.entries = plan->d_entries;
-    a.lpt = plan->d_lpt;
+    thd::FwdArgs a;   // the forward tables, as thd_cp_attn_fwd
+    a.qtiles = plan->d_fqtiles;
+    a.entries = plan->d_fentries;
+    a.lpt = plan->d_flpt;
     a.rm_of_global = plan->d_rm_of_global;
     a.o = static_cast<__nv_bfloat16*>(o_rm);
     a.lse = lse_rm;
@@ -400,7 +416,8 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = plan->d_status;
     if (items == 0) return THD_OK;
-    return thd::launch_fwd_mla_sm100(mq, mkn, mkr, mv, a, (int)items, static_cast<cudaStream_t>(stream))
+    return thd::launch_fwd_mla_sm100(mq, mkn, mkr, mv, mqg, mkng, mkrg, mvg, a, (int)items,
+                                     static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;
 }
@@ -503,8 +520,17 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     a.kt_off = plan->d_kt_off;
     a.kt_list = plan->d_kt_list;
     a.kt_lpt = plan->d_kt_lpt;
-    a.kt_seg = plan->d_kt_seg;
-    a.n_kseg = (int32_t)(plan->kt_seg.size() - 1);
+    a.fqtiles = plan->d_fqtiles;
+    a.fentries = plan->d_fentries;
+    a.fkt_off = plan->d_fkt_off;
+    a.fkt_list = plan->d_fkt_list;
+    a.fkt_lpt = plan->d_fkt_lpt;
+    a.fkt_seg = plan->d_fkt_seg;
+    a.n_fkseg = (int32_t)(plan->fkt_seg.size() - 1);
+    a.rm_of_global = plan->d_rm_of_global;
+    a.q = static_cast<const __nv_bfloat16*>(q_rm);
+    a.k = static_cast<const __nv_bfloat16*>(k_rm);
+    a.v = static_cast<const __nv_bfloat16*>(v_rm);
     a.o = static_cast<const __nv_bfloat16*>(o_rm);
     a.dout = static_cast<const __nv_bfloat16*>(do_rm);
     a.lse = lse_rm;
@@ -520,7 +546,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     a.status = plan->d_status;
     const int64_t nkt = plan->n_qtiles();
     if (nkt == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, plan->kt_seg.back(), num_sms_current(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, plan->fkt_seg.back(), num_sms_current(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

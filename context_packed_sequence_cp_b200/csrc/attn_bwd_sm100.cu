@@ -54,12 +54,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 struct StepMeta {
     int row0, m, qpos0, qbrk, qjump, nvalid, cls;
 };
-__device__ __forceinline__ StepMeta load_meta(const BwdArgs& a, int list_pos) {
-    const int2 pr = __ldg(reinterpret_cast<const int2*>(a.kt_list) + list_pos);
-    const int4 q = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12));      // r, d, row0, m
-    const int4 q2 = __ldg(reinterpret_cast<const int4*>(a.qtiles + (size_t)pr.x * 12) + 1); // qpos0, qbrk, qjump, -
-    const int4 e0 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8));     // k0, nvalid, -, -
-    const int4 e1 = __ldg(reinterpret_cast<const int4*>(a.entries + (size_t)pr.y * 8) + 1); // kjump, cls, -, -
+__device__ __forceinline__ StepMeta load_meta(const int32_t* kt_list, const int32_t* qtiles, const int32_t* entries,
+                                              int list_pos) {
+    const int2 pr = __ldg(reinterpret_cast<const int2*>(kt_list) + list_pos);
+    const int4 q = __ldg(reinterpret_cast<const int4*>(qtiles + (size_t)pr.x * 12));      // r, d, row0, m
+    const int4 q2 = __ldg(reinterpret_cast<const int4*>(qtiles + (size_t)pr.x * 12) + 1); // qpos0, qbrk, qjump, -
+    const int4 e0 = __ldg(reinterpret_cast<const int4*>(entries + (size_t)pr.y * 8));     // k0, nvalid, -, -
+    const int4 e1 = __ldg(reinterpret_cast<const int4*>(entries + (size_t)pr.y * 8) + 1); // kjump, cls, -, -
     StepMeta mt;
     mt.row0 = q.z;
     mt.m = q.w;
@@ -208,13 +209,13 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
             }
         }
-        StepMeta cur = load_meta(a, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        StepMeta cur = load_meta(a.kt_list, a.qtiles, a.entries, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + 1);
         for (int it = 0; it < n_it; ++it) {
             const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
             if (hh == 0 && it > 0) {
                 cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+                if (pos + 1 < llen) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + pos + 1);
             }
             const int h = g * group + hh;
             const int row0 = cur.row0;
@@ -320,14 +321,14 @@ dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale_log2;
         const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
-        StepMeta cur = load_meta(a, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        StepMeta cur = load_meta(a.kt_list, a.qtiles, a.entries, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + 1);
         for (int it = 0; it < n_it; ++it) {
             const int ds = it & 1;
             const int pos = it / group, hh = it - pos * group;
             if (hh == 0 && it > 0) {
                 cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+                if (pos + 1 < llen) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + pos + 1);
             }
             const int m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
             // visible query columns of this key row: a suffix [lo, hi) of the tile
@@ -707,7 +708,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
-                 const __grid_constant__ CUtensorMap tmDV, BwdArgs a) {
+                 const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmQg,
+                 const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmVg,
+                 const __grid_constant__ CUtensorMap tmDOg, BwdArgs a) {
     using L = FusedLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -723,23 +726,30 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // group g.  Items run groups outermost, then segment, then key tiles longest-first:
     // the resident CTAs walk the same THD_KSEG query tiles of a document, so the dQ tiles
     // they add into stay in L2 while they are hot.
-    const int per_group = a.kt_seg[a.n_kseg];
+    // The forward tables: a tile (query or key) is rank-major (row0 >= 0: 128 consecutive
+    // rank-major rows, TMA boxes) or a position tile of a short-chunk document (row0 < 0:
+    // positions pos0 .., rows gathered through rm_of_global with tile::gather4, outputs
+    // added row by row).
+    const int32_t* qtiles = a.fqtiles;
+    const int32_t* entries = a.fentries;
+    const int32_t* kt_list = a.fkt_list;
+    const int per_group = a.fkt_seg[a.n_fkseg];
     const int g = blockIdx.x / per_group;
     const int item = blockIdx.x - g * per_group;
     int seg = 0;
     {
-        int hi = a.n_kseg;  // kt_seg[seg] <= item < kt_seg[hi]
+        int hi = a.n_fkseg;  // fkt_seg[seg] <= item < fkt_seg[hi]
         while (hi - seg > 1) {
             const int mid = (seg + hi) >> 1;
-            if (__ldg(a.kt_seg + mid) <= item) seg = mid;
+            if (__ldg(a.fkt_seg + mid) <= item) seg = mid;
             else hi = mid;
         }
     }
-    const int kt = a.kt_lpt[item - a.kt_seg[seg]];
-    const int* KT = a.qtiles + (size_t)kt * 12;
-    const int k0 = KT[2], kn = KT[3];
-    const int l0 = a.kt_off[kt] + seg * THD_KSEG;
-    const int llen = min(THD_KSEG, a.kt_off[kt + 1] - l0);
+    const int kt = a.fkt_lpt[item - a.fkt_seg[seg]];
+    const int* KT = qtiles + (size_t)kt * 12;
+    const int k0 = KT[2], kn = KT[3], kpos0 = KT[4];
+    const int l0 = a.fkt_off[kt] + seg * THD_KSEG;
+    const int llen = min(THD_KSEG, a.fkt_off[kt + 1] - l0);
     const int n_it = group * llen;
 
     if (threadIdx.x == 0) {
@@ -775,6 +785,18 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (warp == 0) {
         // ---------------------------------------------------- producer warp
         const float log2e = 1.4426950408889634f;
+        // rank-major rows of this lane's 4 rows (4 lane .. 4 lane + 3) of a position tile,
+        // rows past n repeating row n-1
+        auto position_rows = [&](int pos0, int n, int (&rr)[4]) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1));
+        };
+        auto gather = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int heads, int head) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                tma_gather4(map, dst + c * kBox + lane * 512, bar, c * 64, rr[0] * heads + head, rr[1] * heads + head,
+                            rr[2] * heads + head, rr[3] * heads + head);
+        };
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
@@ -783,29 +805,48 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tma_prefetch_desc(&tmDQ);
             tma_prefetch_desc(&tmDK);
             tma_prefetch_desc(&tmDV);
-            const uint32_t kvf = smem_u32(&bars->kv_full);
-            mbar_arrive_expect_tx(kvf, 2 * kTile);
-            for (int c = 0; c < 2; ++c) {
-                tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
-                tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
-            }
         }
-        StepMeta cur = load_meta(a, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        const uint32_t kvf = smem_u32(&bars->kv_full);
+        if (lane == 0) mbar_arrive_expect_tx(kvf, 2 * kTile);
+        __syncwarp();
+        if (k0 >= 0) {
+            if (lane == 0)
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
+                    tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
+                }
+        } else {
+            int rk[4];
+            position_rows(kpos0, kn, rk);
+            gather(&tmKg, sK, kvf, rk, a.hkv, g);
+            gather(&tmVg, sV, kvf, rk, a.hkv, g);
+        }
+        StepMeta cur = load_meta(kt_list, qtiles, entries, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(kt_list, qtiles, entries, l0 + 1);
+        int rq[4] = {0, 0, 0, 0};   // gathered rows of the current query tile (position tiles)
+        int rs[4] = {0, 0, 0, 0};   // rank-major rows of lse / Delta entries lane + 32 u (-1: none)
         for (int it = 0; it < n_it; ++it) {
             const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
             if (hh == 0 && it > 0) {
                 cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+                if (pos + 1 < llen) nxt = load_meta(kt_list, qtiles, entries, l0 + pos + 1);
             }
             const int h = g * group + hh;
             const int row0 = cur.row0;
+            if (hh == 0) {   // rows of a new query tile
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int t = lane + 32 * u;
+                    rs[u] = row0 >= 0 ? (row0 + t < a.T ? row0 + t : -1)
+                                      : (t < cur.m ? __ldg(a.rm_of_global + cur.qpos0 + t) : -1);
+                }
+                if (row0 < 0) position_rows(cur.qpos0, cur.m, rq);
+            }
             float lv[4], dv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int64_t row = (int64_t)row0 + lane + 32 * u;
-                lv[u] = row < a.T ? __ldg(a.lse + (int64_t)h * a.T + row) * log2e : 0.f;
-                dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
+                lv[u] = rs[u] >= 0 ? __ldg(a.lse + (int64_t)h * a.T + rs[u]) * log2e : 0.f;
+                dv[u] = rs[u] >= 0 ? __ldg(a.delta + (int64_t)h * a.T + rs[u]) : 0.f;
             }
             const int st = it & 1;
             // dO(it) refills the stage c(it-2) read: c(it-2) is issued before a(it-1).
@@ -814,9 +855,13 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 mbar_wait(smem_u32(&bars->stat_free[st]), ((it >> 1) - 1) & 1, abort, a.status, 62);
             }
             const uint32_t f = smem_u32(&bars->do_full[st]);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(f, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
+            if (lane == 0) mbar_arrive_expect_tx(f, kTile);
+            __syncwarp();
+            if (row0 >= 0) {
+                if (lane == 0)
+                    for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
+            } else {
+                gather(&tmDOg, sDO + st * kTile, f, rq, a.hq, h);
             }
             float* stat = s_stat + st * 256;
 #pragma unroll
@@ -827,10 +872,14 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             mbar_arrive(f);
             // Q(it) refills the stage d(it-2) read: d(it-2) is issued before e(it-2).
             if (it >= 2) mbar_wait(smem_u32(&bars->dq_full), (it - 2) & 1, abort, a.status, 63);
-            if (lane == 0) {
-                const uint32_t qf = smem_u32(&bars->q_full[st]);
-                mbar_arrive_expect_tx(qf, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, qf, c * 64, h, row0);
+            const uint32_t qf = smem_u32(&bars->q_full[st]);
+            if (lane == 0) mbar_arrive_expect_tx(qf, kTile);
+            __syncwarp();
+            if (row0 >= 0) {
+                if (lane == 0)
+                    for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, qf, c * 64, h, row0);
+            } else {
+                gather(&tmQg, sQ + st * kTile, qf, rq, a.hq, h);
             }
         }
     } else if (warp == 1) {
@@ -917,8 +966,8 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
         // this thread's 128-byte row of dS^T: box hf, row r, 16-byte chunks swizzled by r % 8
         const uint32_t ds_row = sDS + hf * kBox + r * 128;
-        StepMeta cur = load_meta(a, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a, l0 + 1);
+        StepMeta cur = load_meta(kt_list, qtiles, entries, l0), nxt = cur;
+        if (llen > 1) nxt = load_meta(kt_list, qtiles, entries, l0 + 1);
         StepMeta prev = cur;  // the step whose dQ is drained
         int prev_h = 0;
         // Partial sums leave the CTA through its warps: a warp holds 32 rows x 64 columns
@@ -937,16 +986,18 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                              __float_as_uint(__uint_as_float(v[4 * c + 2]) * mul),
                              __float_as_uint(__uint_as_float(v[4 * c + 3]) * mul));
         };
-        // adds the staged box at (row0 + 32 wq, head, col) of a [rows, heads, 128] fp32
-        // tensor with `valid` rows from row0 on
         // The staging rows are rewritten only after stage_free(): a box handed to the TMA unit
         // is waited for (read out of shared memory) there, as late as possible.
         auto stage_free = [&]() {
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
         };
-        auto reduce = [&](const CUtensorMap* map, float* gbase, int heads, int head, int row0, int valid, int col) {
-            if (wq * 32 + 32 <= valid) {
+        // adds the staged box at (row0 + 32 wq, head, col) of a [rows, heads, 128] fp32
+        // tensor with `valid` rows from row0 on; a position tile (row0 < 0) adds its rows
+        // (positions pos0 ..) one by one at their rank-major rows
+        auto reduce = [&](const CUtensorMap* map, float* gbase, int heads, int head, int row0, int pos0, int valid,
+                          int col) {
+            if (row0 >= 0 && wq * 32 + 32 <= valid) {
                 fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
                 __syncwarp();
                 if (lane == 0) {
@@ -962,8 +1013,8 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     const int q = wq * 32 + rr;
                     if (q < valid) {
                         const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
-                        red_add_v4(gbase + ((int64_t)(row0 + q) * heads + head) * kD + col + 4 * chunk, x.x, x.y,
-                                   x.z, x.w);
+                        const int row = row0 >= 0 ? row0 + q : __ldg(a.rm_of_global + pos0 + q);
+                        red_add_v4(gbase + ((int64_t)row * heads + head) * kD + col + 4 * chunk, x.x, x.y, x.z, x.w);
                     }
                 }
                 __syncwarp();
@@ -982,17 +1033,17 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
-            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.m, hf * 64);
+            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             stage_free();
             stage(v, a.scale);
-            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.m, hf * 64 + 32);
+            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
         };
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
             const int pos = it / group, hh = it - pos * group;
             if (hh == 0 && it > 0) {
                 cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a, l0 + pos + 1);
+                if (pos + 1 < llen) nxt = load_meta(kt_list, qtiles, entries, l0 + pos + 1);
             }
             const int m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
             // visible query columns of this key row: a suffix [lo, hi) of the tile
@@ -1092,7 +1143,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tmem_wait_ld();
                 stage_free();
                 stage(v, which == 0 ? a.scale : 1.f);
-                reduce(which == 0 ? &tmDK : &tmDV, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kn, hf * 64 + ch * 32);
+                reduce(which == 0 ? &tmDK : &tmDV, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kpos0, kn, hf * 64 + ch * 32);
             }
         }
         stage_free();   // every box read before the CTA's shared memory is released
@@ -1116,15 +1167,18 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
     if (fused) {
         static std::atomic<uint64_t> fused_configured{0};
         if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, fused_configured)) return -1;
-        CUtensorMap mdq, mdk, mdv;
+        CUtensorMap mdq, mdk, mdv, mqg, mkg, mvg, mdog;
         if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&mdk, a.dk, a.T, a.hkv, kD) ||
-            !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD))
+            !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&mqg, a.q, a.T * a.hq, kD) ||
+            !make_map_bf16_rows(&mkg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&mvg, a.v, a.T * a.hkv, kD) ||
+            !make_map_bf16_rows(&mdog, a.dout, a.T * a.hq, kD))
             return -1;
         bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.dk, a.dv, a.T * a.hkv,
                                                          a.T * a.hq, a.hq, a.T);
         if (cudaGetLastError() != cudaSuccess) return -1;
         const unsigned items = (unsigned)((int64_t)n_items_per_group * a.hkv);
-        bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, a);
+        bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, mqg, mkg,
+                                                                           mvg, mdog, a);
         return cudaGetLastError() == cudaSuccess ? 0 : -1;
     }
     static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKr,
            const __grid_constant__ CUtensorMap tmQg, const __grid_constant__ CUtensorMap tmKg,
-           const __grid_constant__ CUtensorMap tmVg, FwdArgs a) {
+           const __grid_constant__ CUtensorMap tmVg, const __grid_constant__ CUtensorMap tmKrg, FwdArgs a) {
     static_assert(!SHARED_ROPE || DQK == 192, "the shared rope key is the third 64-column box");
     using L = FwdLayout<DQK, DV>;
     constexpr int NK = L::NK, NV = L::NV;
@@ -160,15 +160,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // rm_of_global: every lane gathers 4 rows per 64-column box (tile::gather4), rows
         // past n repeat row n-1 (they are masked).
         const bool is_k = warp == 0;
-        // this lane's 4 rows of a position tile (their indices are loaded one tile ahead,
-        // so that the load latency overlaps the wait for a free stage)
-        auto gather_index = [&](int pos0, int n, int heads, int head, int (&rr)[4]) {
+        // this lane's 4 rank-major rows of a position tile (their indices are loaded one
+        // tile ahead, so that the load latency overlaps the wait for a free stage)
+        auto gather_index = [&](int pos0, int n, int (&rr)[4]) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1)) * heads + head;
+            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1));
         };
-        auto gather_rows = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int nbox) {
-            for (int c = 0; c < nbox; ++c)
-                tma_gather4(map, dst + c * L::kBox + lane * 512, bar, c * 64, rr[0], rr[1], rr[2], rr[3]);
+        // 64-column boxes c0 .. c1-1 of those rows, row (rm * heads + head) of the row map
+        auto gather_rows = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int heads,
+                               int head, int c0, int c1) {
+            for (int c = c0; c < c1; ++c)
+                tma_gather4(map, dst + c * L::kBox + lane * 512, bar, (c - c0) * 64, rr[0] * heads + head,
+                            rr[1] * heads + head, rr[2] * heads + head, rr[3] * heads + head);
         };
         if (is_k) {
             if (lane == 0) {
@@ -182,10 +185,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             if (row0 >= 0) {
                 if (lane == 0)
                     for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, h, row0);
-            } else if (!SHARED_ROPE) {
+            } else {
                 int rq[4];
-                gather_index(qpos0, m, a.hq, h, rq);
-                gather_rows(&tmQg, sQ, qf, rq, DQK / 64);
+                gather_index(qpos0, m, rq);
+                gather_rows(&tmQg, sQ, qf, rq, a.hq, h, 0, DQK / 64);
             }
         } else if (lane == 0) {
             tma_prefetch_desc(&tmV);
@@ -193,14 +196,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int ns = is_k ? NK : NV;
         int4 e_next = nk > 0 ? __ldg(reinterpret_cast<const int4*>(E)) : make_int4(0, 0, 0, 0);
         int rr_next[4] = {0, 0, 0, 0};
-        if (!SHARED_ROPE && nk > 0 && e_next.x < 0) gather_index(e_next.z, e_next.y, a.hkv, g, rr_next);
+        if (nk > 0 && e_next.x < 0) gather_index(e_next.z, e_next.y, rr_next);
         for (int j = 0; j < nk; ++j) {
             const int st = j % ns;
             const int4 e = e_next;   // k0, nvalid, kpos0, -
             int rr[4] = {rr_next[0], rr_next[1], rr_next[2], rr_next[3]};
             if (j + 1 < nk) {
                 e_next = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
-                if (!SHARED_ROPE && e_next.x < 0) gather_index(e_next.z, e_next.y, a.hkv, g, rr_next);
+                if (e_next.x < 0) gather_index(e_next.z, e_next.y, rr_next);
             }
             // A stage is refilled once the MMA that read it has retired: K_{j-NK} is
             // read by S_{j-NK} (signalled on s_full), V_{j-NV} by PV_{j-NV} (o_done).
@@ -220,8 +223,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                             else
                                 tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, e.x);
                         }
-                } else if (!SHARED_ROPE) {
-                    gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, DQK / 64);
+                } else if (SHARED_ROPE) {   // per-head part, then the shared rope key (one row per token)
+                    gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, a.hkv, g, 0, 2);
+                    gather_rows(&tmKrg, sK + st * L::kKBytes, kf, rr, 1, 0, 2, 3);
+                } else {
+                    gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, a.hkv, g, 0, DQK / 64);
                 }
             } else {
                 if (j >= NV)
@@ -233,8 +239,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     if (lane == 0)
                         for (int c = 0; c < DV / 64; ++c)
                             tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, e.x);
-                } else if (!SHARED_ROPE) {
-                    gather_rows(&tmVg, sV + st * L::kVBytes, vf, rr, DV / 64);
+                } else {
+                    gather_rows(&tmVg, sV + st * L::kVBytes, vf, rr, a.hkv, g, 0, DV / 64);
                 }
             }
         }
@@ -441,12 +447,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
 template <int DQK, int DV, bool SHARED_ROPE>
 int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr,
-           const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a, int n_items,
-           cudaStream_t stream) {
+           const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const CUtensorMap& krg,
+           const FwdArgs& a, int n_items, cudaStream_t stream) {
     using L = FwdLayout<DQK, DV>;
     static std::atomic<uint64_t> configured{0};
     if (!ensure_dynamic_smem(fwd_kernel<DQK, DV, SHARED_ROPE>, L::kDynSmem, configured)) return -1;
-    fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, qg, kg, vg, a);
+    fwd_kernel<DQK, DV, SHARED_ROPE><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, qg, kg, vg, krg, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -455,16 +461,16 @@ int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, con
 int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a,
                      int n_items, cudaStream_t stream) {
-    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, qg, kg, vg, a, n_items, stream);
-    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, qg, kg, vg, a, n_items, stream);
+    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, qg, kg, vg, kg, a, n_items, stream);
+    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, qg, kg, vg, kg, a, n_items, stream);
     return -2;
 }
 
-// The compact-key form walks rank-major tiles only (the tables it is given have no
-// position tiles), so its row maps are never read.
 int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
-                         const CUtensorMap& v, const FwdArgs& a, int n_items, cudaStream_t stream) {
-    return launch<192, 128, true>(q, k_nope, v, k_rope, q, k_nope, v, a, n_items, stream);
+                         const CUtensorMap& v, const CUtensorMap& qg, const CUtensorMap& k_nope_g,
+                         const CUtensorMap& k_rope_g, const CUtensorMap& vg, const FwdArgs& a, int n_items,
+                         cudaStream_t stream) {
+    return launch<192, 128, true>(q, k_nope, v, k_rope, qg, k_nope_g, vg, k_rope_g, a, n_items, stream);
 }
 
 }  // namespace thd

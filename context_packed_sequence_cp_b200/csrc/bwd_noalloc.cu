@@ -87,8 +87,17 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     a.kt_off = plan->d_kt_off;
     a.kt_list = plan->d_kt_list;
     a.kt_lpt = plan->d_kt_lpt;
-    a.kt_seg = plan->d_kt_seg;
-    a.n_kseg = (int32_t)(plan->kt_seg.size() - 1);
+    a.fqtiles = plan->d_fqtiles;
+    a.fentries = plan->d_fentries;
+    a.fkt_off = plan->d_fkt_off;
+    a.fkt_list = plan->d_fkt_list;
+    a.fkt_lpt = plan->d_fkt_lpt;
+    a.fkt_seg = plan->d_fkt_seg;
+    a.n_fkseg = (int32_t)(plan->fkt_seg.size() - 1);
+    a.rm_of_global = plan->d_rm_of_global;
+    a.q = static_cast<const __nv_bfloat16*>(q_rm);
+    a.k = static_cast<const __nv_bfloat16*>(k_rm);
+    a.v = static_cast<const __nv_bfloat16*>(v_rm);
     a.o = static_cast<const __nv_bfloat16*>(o_rm);
     a.dout = static_cast<const __nv_bfloat16*>(do_rm);
     a.lse = lse_rm;
@@ -103,7 +112,7 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = plan->d_status;
     if (plan->n_qtiles() == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)plan->n_qtiles(), plan->kt_seg.back(), sm_count(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)plan->n_qtiles(), plan->fkt_seg.back(), sm_count(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

@@ -60,7 +60,9 @@ int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
 // Multi-head latent attention with a shared rope key: Q [T, hq, 192], K_nope [T, hkv, 128],
 // K_rope [T, 1, 64] (one per token, every head), V [T, hkv, 128].
 int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
-                         const CUtensorMap& v, const FwdArgs& a, int n_items, cudaStream_t stream);
+                         const CUtensorMap& v, const CUtensorMap& qg, const CUtensorMap& k_nope_g,
+                         const CUtensorMap& k_rope_g, const CUtensorMap& vg, const FwdArgs& a, int n_items,
+                         cudaStream_t stream);
 
 // ---- forward, fp32 SIMT --------------------------------------------------------
 struct FwdF32Args {
@@ -86,8 +88,19 @@ struct BwdArgs {
     const int32_t* kt_off;
     const int32_t* kt_list;
     const int32_t* kt_lpt;
-    const int32_t* kt_seg;  // backward work items by list segment (THD_KSEG entries each)
-    int32_t n_kseg;
+    // the fused kernel walks the forward tables (rank-major and position tiles) and their
+    // key-tile transpose; position rows are found through rm_of_global
+    const int32_t* fqtiles;
+    const int32_t* fentries;
+    const int32_t* fkt_off;
+    const int32_t* fkt_list;
+    const int32_t* fkt_lpt;
+    const int32_t* fkt_seg;  // work items by list segment (THD_KSEG entries each)
+    int32_t n_fkseg;
+    const int32_t* rm_of_global;
+    const __nv_bfloat16* q;     // rank-major inputs (row maps of the position tiles)
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;
     const float* lse;

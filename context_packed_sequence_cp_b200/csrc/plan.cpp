@@ -64,6 +64,56 @@ struct Layout {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Key-tile transpose of a tile table (entries name their key tile in field 6, an index
+// into the same tile table): per key tile the (query tile, entry) pairs, in descending
+// order of the query tile's last position, ties (which cannot occur within one
+// document) by tile index.  A key tile sees exactly the query tiles of its document
+// whose last position is at or past its first key, so every list is a prefix of one
+// per-document order, and key tiles walked at the same time read the same query tiles.
+// Walking the query tiles once in that order makes the counting-sort fill emit every
+// list already sorted.  Also the longest-first order of key tiles and the work items
+// per list segment (segment j of every key tile whose list reaches it: the first n_j
+// key tiles of the longest-first order).
+void build_transpose(const std::vector<int32_t>& qtiles, const std::vector<int32_t>& entries,
+                     std::vector<int32_t>& kt_off, std::vector<int32_t>& kt_list, std::vector<int32_t>& kt_lpt,
+                     std::vector<int32_t>& kt_seg) {
+    const int64_t n_tiles = (int64_t)qtiles.size() / THD_QTILE_FIELDS;
+    const int64_t ne = (int64_t)entries.size() / THD_ENTRY_FIELDS;
+    kt_off.assign(n_tiles + 1, 0);
+    for (int64_t e = 0; e < ne; ++e) kt_off[entries[(size_t)e * THD_ENTRY_FIELDS + 6] + 1]++;
+    for (int64_t t = 0; t < n_tiles; ++t) kt_off[t + 1] += kt_off[t];
+    std::vector<int32_t> by_last(n_tiles);
+    for (int64_t t = 0; t < n_tiles; ++t) by_last[t] = (int32_t)t;
+    std::sort(by_last.begin(), by_last.end(), [&](int32_t a, int32_t b) {
+        const int32_t pa = qtiles[(size_t)a * THD_QTILE_FIELDS + 7];
+        const int32_t pb = qtiles[(size_t)b * THD_QTILE_FIELDS + 7];
+        return pa != pb ? pa > pb : a < b;
+    });
+    std::vector<int32_t> fill(kt_off.begin(), kt_off.end() - 1);
+    kt_list.assign((size_t)ne * 2, 0);
+    for (const int32_t qt : by_last) {
+        const int32_t* q = &qtiles[(size_t)qt * THD_QTILE_FIELDS];
+        for (int64_t e = q[9]; e < (int64_t)q[9] + q[8]; ++e) {
+            const int32_t kt = entries[(size_t)e * THD_ENTRY_FIELDS + 6];
+            const int32_t at = fill[kt]++;
+            kt_list[(size_t)at * 2] = qt;
+            kt_list[(size_t)at * 2 + 1] = (int32_t)e;
+        }
+    }
+    kt_lpt.resize(n_tiles);
+    for (int64_t t = 0; t < n_tiles; ++t) kt_lpt[t] = (int32_t)t;
+    std::stable_sort(kt_lpt.begin(), kt_lpt.end(),
+                     [&](int32_t a, int32_t b) { return kt_off[a + 1] - kt_off[a] > kt_off[b + 1] - kt_off[b]; });
+    const int64_t max_len = n_tiles ? (int64_t)kt_off[kt_lpt[0] + 1] - kt_off[kt_lpt[0]] : 0;
+    const int64_t n_seg = ceil_div(max_len, THD_KSEG);
+    kt_seg.assign(n_seg + 1, 0);
+    int64_t reach = n_tiles;  // key tiles whose list is longer than j * THD_KSEG
+    for (int64_t j = 0; j < n_seg; ++j) {
+        while (reach > 0 && (int64_t)kt_off[kt_lpt[reach - 1] + 1] - kt_off[kt_lpt[reach - 1]] <= j * THD_KSEG) --reach;
+        kt_seg[j + 1] = (int32_t)(kt_seg[j] + reach);
+    }
+}
+
 }  // namespace
 
 int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s* p) {
@@ -179,53 +229,8 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
             return p->qtiles[(size_t)a * THD_QTILE_FIELDS + 8] > p->qtiles[(size_t)b * THD_QTILE_FIELDS + 8];
         });
 
-        // ---- key-tile transpose for the backward (counting sort by key tile) --
-        // Each key tile's list is in descending order of the query tile's last
-        // position, ties (which cannot occur within one document) by tile index.  A
-        // key tile sees exactly the query tiles of its document whose last position is
-        // at or past its first key, so every list is a prefix of one per-document
-        // order, and key tiles walked at the same time read the same query tiles.
-        // Walking the query tiles once in that order makes the counting-sort fill
-        // emit every list already sorted.
-        const int64_t ne = n_entries;
-        p->kt_off.assign(n_tiles + 1, 0);
-        for (int64_t e = 0; e < ne; ++e) p->kt_off[p->entries[(size_t)e * THD_ENTRY_FIELDS + 6] + 1]++;
-        for (int64_t t = 0; t < n_tiles; ++t) p->kt_off[t + 1] += p->kt_off[t];
-        std::vector<int32_t> by_last(n_tiles);
-        for (int64_t t = 0; t < n_tiles; ++t) by_last[t] = (int32_t)t;
-        std::sort(by_last.begin(), by_last.end(), [&](int32_t a, int32_t b) {
-            const int32_t pa = p->qtiles[(size_t)a * THD_QTILE_FIELDS + 7];
-            const int32_t pb = p->qtiles[(size_t)b * THD_QTILE_FIELDS + 7];
-            return pa != pb ? pa > pb : a < b;
-        });
-        std::vector<int32_t> fill(p->kt_off.begin(), p->kt_off.end() - 1);
-        p->kt_list.assign((size_t)ne * 2, 0);
-        for (const int32_t qt : by_last) {
-            const int32_t* q = &p->qtiles[(size_t)qt * THD_QTILE_FIELDS];
-            for (int64_t e = q[9]; e < (int64_t)q[9] + q[8]; ++e) {
-                const int32_t kt = p->entries[(size_t)e * THD_ENTRY_FIELDS + 6];
-                const int32_t at = fill[kt]++;
-                p->kt_list[(size_t)at * 2] = qt;
-                p->kt_list[(size_t)at * 2 + 1] = (int32_t)e;
-            }
-        }
-        p->kt_lpt.resize(n_tiles);
-        for (int64_t t = 0; t < n_tiles; ++t) p->kt_lpt[t] = (int32_t)t;
-        std::stable_sort(p->kt_lpt.begin(), p->kt_lpt.end(), [&](int32_t a, int32_t b) {
-            return p->kt_off[a + 1] - p->kt_off[a] > p->kt_off[b + 1] - p->kt_off[b];
-        });
-        // Backward work items: segment j of every key tile whose list reaches it.  kt_lpt
-        // is by descending list length, so those key tiles are its first n_j entries.
-        const int64_t max_len = n_tiles ? (int64_t)p->kt_off[p->kt_lpt[0] + 1] - p->kt_off[p->kt_lpt[0]] : 0;
-        const int64_t n_seg = ceil_div(max_len, THD_KSEG);
-        p->kt_seg.assign(n_seg + 1, 0);
-        int64_t reach = n_tiles;  // key tiles whose list is longer than j * THD_KSEG
-        for (int64_t j = 0; j < n_seg; ++j) {
-            while (reach > 0 && (int64_t)p->kt_off[p->kt_lpt[reach - 1] + 1] - p->kt_off[p->kt_lpt[reach - 1]] <=
-                                    j * THD_KSEG)
-                --reach;
-            p->kt_seg[j + 1] = (int32_t)(p->kt_seg[j] + reach);
-        }
+        // ---- key-tile transpose for the backward ----------------------------
+        build_transpose(p->qtiles, p->entries, p->kt_off, p->kt_list, p->kt_lpt, p->kt_seg);
 
         // ---- forward tables -------------------------------------------------
         // A document whose chunks are shorter than a tile (c < BM) puts two or more
@@ -235,20 +240,30 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         // s + v*BM .. (read in place from the rank-major buffers through rm_of_global),
         // key tiles 0 .. u listed for query tile u, the last one the diagonal.  Rank-major
         // records are marked by row0 / k0 >= 0; position records carry -1 there.
+        // An entry's key tile (field 6) is the forward tile that holds its keys.
         p->fqtiles.clear();
         p->fentries.clear();
+        std::vector<int32_t> f_of_tile(n_tiles, -1);  // forward index of a rank-major tile
+        int32_t nf_rm = 0;
+        for (int64_t t = 0; t < n_tiles; ++t)
+            if (lay.chunk(p->qtiles[(size_t)t * THD_QTILE_FIELDS + 1]) >= BM) f_of_tile[t] = nf_rm++;
         for (int64_t t = 0; t < n_tiles; ++t) {
             const int32_t* q = &p->qtiles[(size_t)t * THD_QTILE_FIELDS];
-            if (lay.chunk(q[1]) < BM) continue;
+            if (f_of_tile[t] < 0) continue;
             const int32_t off = (int32_t)(p->fentries.size() / THD_ENTRY_FIELDS);
             p->fqtiles.insert(p->fqtiles.end(), q, q + THD_QTILE_FIELDS);
             p->fqtiles[p->fqtiles.size() - THD_QTILE_FIELDS + 9] = off;
             p->fentries.insert(p->fentries.end(), p->entries.begin() + (size_t)q[9] * THD_ENTRY_FIELDS,
                                p->entries.begin() + (size_t)(q[9] + q[8]) * THD_ENTRY_FIELDS);
+            for (int64_t e = off; e < (int64_t)off + q[8]; ++e) {
+                int32_t& kt = p->fentries[(size_t)e * THD_ENTRY_FIELDS + 6];
+                kt = f_of_tile[kt];
+            }
         }
         for (int d = 0; d < n_docs; ++d) {
             if (lay.chunk(d) >= BM) continue;
             const int64_t n = ceil_div(L[d], BM);
+            const int32_t first_tile = (int32_t)(p->fqtiles.size() / THD_QTILE_FIELDS);  // position tile 0 of d
             for (int64_t u = 0; u < n; ++u) {
                 const int64_t p0 = s[d] + u * BM, m = std::min<int64_t>(BM, L[d] - u * BM), qmax = p0 + m - 1;
                 const int32_t rec[THD_QTILE_FIELDS] = {-1, d, -1, (int32_t)m, (int32_t)p0, (int32_t)m, 0, (int32_t)qmax,
@@ -259,7 +274,8 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
                 for (int64_t v = 0; v <= u; ++v) {
                     const int64_t kp0 = s[d] + v * BM, nv = std::min<int64_t>(BM, qmax - kp0 + 1);
                     const int32_t cls = kp0 + nv - 1 <= p0 ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
-                    const int32_t e[THD_ENTRY_FIELDS] = {-1, (int32_t)nv, (int32_t)kp0, (int32_t)nv, 0, cls, -1, -1};
+                    const int32_t e[THD_ENTRY_FIELDS] = {-1, (int32_t)nv, (int32_t)kp0, (int32_t)nv, 0, cls,
+                                                         first_tile + (int32_t)v, -1};
                     p->fentries.insert(p->fentries.end(), e, e + THD_ENTRY_FIELDS);
                 }
             }
@@ -270,6 +286,8 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         std::stable_sort(p->flpt.begin(), p->flpt.end(), [&](int32_t a, int32_t b) {
             return p->fqtiles[(size_t)a * THD_QTILE_FIELDS + 8] > p->fqtiles[(size_t)b * THD_QTILE_FIELDS + 8];
         });
+        // the fused backward walks the forward tables, key tile by key tile
+        build_transpose(p->fqtiles, p->fentries, p->fkt_off, p->fkt_list, p->fkt_lpt, p->fkt_seg);
     } catch (const std::bad_alloc&) {
         return THD_ERR_ALLOC;
     }

@@ -21,6 +21,7 @@ struct thd_cp_plan_s {
     // forward tables: rank-major tiles of documents whose chunks span a tile or more,
     // position-ordered tiles of documents with shorter chunks
     std::vector<int32_t> fqtiles, fentries, flpt;
+    std::vector<int32_t> fkt_off, fkt_list, fkt_lpt, fkt_seg;  // their key-tile transpose
 
     // Device side, valid after thd_cp_plan_upload.  Every table lives in one
     // stream-ordered allocation (d_buf, grown only when a layout needs more), and
@@ -38,6 +39,7 @@ struct thd_cp_plan_s {
     int32_t *d_qtiles = nullptr, *d_entries = nullptr, *d_lpt = nullptr;
     int32_t *d_kt_off = nullptr, *d_kt_list = nullptr, *d_kt_lpt = nullptr, *d_kt_seg = nullptr;
     int32_t *d_fqtiles = nullptr, *d_fentries = nullptr, *d_flpt = nullptr;
+    int32_t *d_fkt_off = nullptr, *d_fkt_list = nullptr, *d_fkt_lpt = nullptr, *d_fkt_seg = nullptr;
     int32_t* d_status = nullptr;  // set by kernels whose bounded waits gave up
 
     int64_t n_qtiles() const { return (int64_t)qtiles.size() / THD_QTILE_FIELDS; }

@@ -85,6 +85,7 @@ typedef struct thd_cp_plan_info_s {
     int64_t n_kseg;     /* segments of the longest key-tile list (THD_KSEG entries each) */
     int64_t n_fqtiles;  /* query tiles of the forward tables (thd_cp_plan_export_fwd)   */
     int64_t n_fentries; /* entries of the forward tables                                */
+    int64_t n_fkseg;    /* segments of the longest key-tile list of the forward tables  */
 } thd_cp_plan_info_t;
 
 /*
@@ -205,13 +206,18 @@ int thd_cp_plan_export(thd_cp_plan_t plan, int32_t* q_idx, int32_t* rm_of_global
  *             short-chunk document d (ascending) and u = 0 .. ceil(L/128)-1, a position
  *             tile: r = -1, d, row0 = -1, m = min(128, L - 128u), qpos0 = s_d + 128u,
  *             qbrk = m, qjump = 0, qpos_max, nk = u + 1, entry_off, doc_start, doc_end.
- *   fentries  int32[n_fentries * 8], entry layout.  For a position tile, its key tiles
- *             v = 0 .. u: k0 = -1, nvalid (128, or m for v = u), kpos0 = s_d + 128v,
- *             kbrk = nvalid, kjump = 0, cls (UNMASKED below the diagonal), ktile = -1,
- *             key_rank = -1.
+ *   fentries  int32[n_fentries * 8], entry layout; ktile (field 6) is the index in
+ *             fqtiles of the tile holding the entry's keys.  For a position tile, its key
+ *             tiles v = 0 .. u: k0 = -1, nvalid (128, or m for v = u), kpos0 = s_d + 128v,
+ *             kbrk = nvalid, kjump = 0, cls (UNMASKED below the diagonal), ktile = the
+ *             position tile v of d, key_rank = -1.
  *   flpt      int32[n_fqtiles]  forward query tiles by descending nk (ties by index).
+ *   fkt_off, fkt_list, fkt_lpt, fkt_seg  the key-tile transpose of these tables, laid
+ *             out as kt_off / kt_list / kt_lpt / kt_seg (sizes n_fqtiles + 1,
+ *             n_fentries * 2, n_fqtiles, n_fkseg + 1): the backward walks it.
  */
-int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt);
+int thd_cp_plan_export_fwd(thd_cp_plan_t plan, int32_t* fqtiles, int32_t* fentries, int32_t* flpt,
+                           int32_t* fkt_off, int32_t* fkt_list, int32_t* fkt_lpt, int32_t* fkt_seg);
 
 /*
  * thd_cp_plan_upload -- copy the tables to the current device once and keep them

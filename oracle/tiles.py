@@ -125,6 +125,24 @@ def tile_plan(cu_seqlens, cp: int) -> dict:
     n_tiles = len(tiles)
     lpt = np.array(sorted(range(n_tiles), key=lambda t: (-int(qtiles[t, 8]), t)), dtype=np.int32)
 
+    kt_off, kt_list, kt_lpt, kt_seg = _transpose(qtiles, entries)
+
+    fqtiles, fentries, flpt = _forward_tables(cu, cp, qtiles, entries)
+    fkt_off, fkt_list, fkt_lpt, fkt_seg = _transpose(fqtiles, fentries)
+    return dict(T=int(cu[-1]), cp=int(cp), Tl=int(cu[-1]) // cp, n_docs=n_docs,
+                q_idx=q_idx, rm_of_global=rm_of_global, qtiles=qtiles, entries=entries,
+                lpt=lpt, kt_off=kt_off, kt_list=kt_list, kt_lpt=kt_lpt, kt_seg=kt_seg,
+                fqtiles=fqtiles, fentries=fentries, flpt=flpt,
+                fkt_off=fkt_off, fkt_list=fkt_list, fkt_lpt=fkt_lpt, fkt_seg=fkt_seg)
+
+
+def _transpose(qtiles, entries):
+    """Per key tile (entry field 6 names it, an index into the same tile table) the
+    list of (q-tile, entry) pairs, by descending last query position, then q-tile index;
+    key tiles by descending list length; and the running count of backward work items
+    per list segment (segment j of every key tile whose list has more than j*KSEG
+    entries)."""
+    n_tiles = qtiles.shape[0]
     lists = [[] for _ in range(n_tiles)]
     for qt in range(n_tiles):
         e0, nk = int(qtiles[qt, 9]), int(qtiles[qt, 8])
@@ -132,22 +150,14 @@ def tile_plan(cu_seqlens, cp: int) -> dict:
             lists[int(entries[e, 6])].append((qt, e))
     kt_off = np.zeros(n_tiles + 1, dtype=np.int32)
     kt_off[1:] = np.cumsum([len(x) for x in lists])
-    # each key tile's list by descending last query position, then q-tile index
     kt_list = np.array([p for x in lists for p in sorted(x, key=lambda pr: (-int(qtiles[pr[0], 7]), pr[0]))],
                        dtype=np.int32).reshape(-1, 2)
     kt_lpt = np.array(sorted(range(n_tiles), key=lambda t: (-len(lists[t]), t)), dtype=np.int32)
-    # backward work items: segment j (entries j*KSEG .. j*KSEG+KSEG-1) of every key tile
-    # whose list is longer than j*KSEG; kt_seg holds their running count per segment
     n_seg = -(-max((len(x) for x in lists), default=0) // KSEG)
     kt_seg = np.zeros(n_seg + 1, dtype=np.int32)
     for j in range(n_seg):
         kt_seg[j + 1] = kt_seg[j] + sum(1 for x in lists if len(x) > j * KSEG)
-
-    fqtiles, fentries, flpt = _forward_tables(cu, cp, qtiles, entries)
-    return dict(T=int(cu[-1]), cp=int(cp), Tl=int(cu[-1]) // cp, n_docs=n_docs,
-                q_idx=q_idx, rm_of_global=rm_of_global, qtiles=qtiles, entries=entries,
-                lpt=lpt, kt_off=kt_off, kt_list=kt_list, kt_lpt=kt_lpt, kt_seg=kt_seg,
-                fqtiles=fqtiles, fentries=fentries, flpt=flpt)
+    return kt_off, kt_list, kt_lpt, kt_seg
 
 
 def _forward_tables(cu, cp, qtiles, entries):
@@ -155,22 +165,26 @@ def _forward_tables(cu, cp, qtiles, entries):
     (L / (2 cp) < 128) is tiled in position order: query tile u holds positions
     s + 128u .. (up to 128), and every key tile v (positions s + 128v ..) holding a key
     that some of its queries can see is listed, found by enumerating the (query, key)
-    pairs; row0 / k0 / r / ktile / key_rank are -1 for these records (the rows are
-    found through rm_of_global).  Other documents keep their rank-major tiles, in the
-    order of the main table, first."""
+    pairs; row0 / k0 / r / key_rank are -1 for these records (the rows are found
+    through rm_of_global).  Other documents keep their rank-major tiles, in the order of
+    the main table, first.  An entry's key tile (field 6) is the index, in these
+    tables, of the tile that holds its keys."""
     n_docs = cu.size - 1
     short = {d for d in range(n_docs) if (int(cu[d + 1]) - int(cu[d])) // (2 * cp) < BM}
+    kept = [t for t in range(qtiles.shape[0]) if int(qtiles[t, 1]) not in short]
+    f_of_tile = {t: i for i, t in enumerate(kept)}      # forward index of a rank-major tile
     fq, fe = [], []
-    for t in range(qtiles.shape[0]):
-        if int(qtiles[t, 1]) in short:
-            continue
+    for t in kept:
         rec = qtiles[t].copy()
         e0, nk = int(rec[9]), int(rec[8])
         rec[9] = len(fe)
         fq.append(rec)
-        fe.extend(entries[e0:e0 + nk].tolist())
+        for en in entries[e0:e0 + nk].tolist():
+            en[6] = f_of_tile[en[6]]                     # key tile: its forward index
+            fe.append(en)
     for d in sorted(short):
         s, e = int(cu[d]), int(cu[d + 1])
+        first_tile = len(fq)                             # position tile 0 of d
         for p0 in range(s, e, BM):
             qpos = np.arange(p0, min(p0 + BM, e))
             first = len(fe)
@@ -183,7 +197,7 @@ def _forward_tables(cu, cp, qtiles, entries):
                     continue
                 assert seen[:nv].all(), "visible keys of a position tile form a prefix"
                 cls = UNMASKED if vis[:, :nv].all() else PARTIAL
-                fe.append([-1, nv, int(kpos[0]), nv, 0, cls, -1, -1])
+                fe.append([-1, nv, int(kpos[0]), nv, 0, cls, first_tile + (k0 - s) // BN, -1])
             fq.append(np.array([-1, d, -1, qpos.size, int(qpos[0]), qpos.size, 0, int(qpos[-1]),
                                 len(fe) - first, first, s, e], dtype=np.int32))
     fqtiles = np.array(fq, dtype=np.int32).reshape(-1, QT_FIELDS)

@@ -177,3 +177,22 @@ def test_bwd_rejects_unsupported():
     with pytest.raises(thd.ThdError) as e:
         thd.thd_cp_attn_bwd(plan, x, x, y, y, lse, y)
     assert e.value.kind == "UNSUPPORTED"
+
+
+@pytest.mark.parametrize("cp", [2, 4])
+def test_bwd_position_tiles_around_the_chunk_threshold(cp):
+    """The backward walks the forward tables: documents whose chunks are shorter than a
+    tile as position tiles (keys, queries and their gradients gathered / added through
+    rm_of_global), the others rank-major; chunk sizes 1, 17, 64, 127 and 128, 129, 300 in
+    one packed sequence, GQA 8/2, every gradient compared."""
+    chunks = [1, 17, 64, 127, 128, 129, 300, 3]
+    cu = syn.cu_seqlens_of([2 * cp * c for c in chunks])
+    T = int(cu[-1])
+    q, k, v, do = syn.make_tensors(T, 8, 2, 128, 128, torch.bfloat16, seed=50 + cp, with_do=True)
+    (dq, dk, dv), plan = run_fwd_bwd(cu, cp, q, k, v, do)
+    assert (plan.export_fwd()["fqtiles"][:, 2] < 0).any()
+    o, lse = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
+    wq, wk, wv = A.attention_bwd(q, k, v, o, lse, do, cu, 1 / math.sqrt(128))
+    assert_bf16_close(dq, wq, "dQ")
+    assert_bf16_close(dk, wk, "dK")
+    assert_bf16_close(dv, wv, "dV")

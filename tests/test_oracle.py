@@ -142,6 +142,9 @@ def test_forward_tables_cover_every_visible_pair_once(seed):
                 kpos = TT.decode_run(int(en[2]), int(en[3]), int(en[4]), int(en[1]))
                 if en[0] >= 0:
                     assert np.array_equal(plan["q_idx"][en[0]:en[0] + en[1]], kpos)
+                # its key tile (a tile of the same tables) starts with the entry's first key
+                kt = plan["fqtiles"][en[6]]
+                assert kt[4] == kpos[0] and kt[1] == d and (kt[2] == en[0] or kt[2] < 0)
                 assert np.all(doc[kpos] == d)
                 vis = kpos[None, :] <= qpos[:, None]
                 cnt = int(vis.sum())

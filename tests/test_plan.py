@@ -10,7 +10,7 @@ from oracle import partition as P
 from oracle import tiles as TT
 
 KEYS = ("q_idx", "rm_of_global", "qtiles", "entries", "lpt", "kt_off", "kt_list", "kt_lpt", "kt_seg")
-FWD_KEYS = ("fqtiles", "fentries", "flpt")
+FWD_KEYS = ("fqtiles", "fentries", "flpt", "fkt_off", "fkt_list", "fkt_lpt", "fkt_seg")
 
 
 def _compare(cu, cp):
