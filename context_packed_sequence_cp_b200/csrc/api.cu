@@ -514,12 +514,6 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
         !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !make_map_bf16(&mdo, do_rm, plan->T, hq, dv))
         return THD_ERR_CUDA;
     thd::BwdArgs a;
-    a.qtiles = plan->d_qtiles;
-    a.entries = plan->d_entries;
-    a.lpt = plan->d_lpt;
-    a.kt_off = plan->d_kt_off;
-    a.kt_list = plan->d_kt_list;
-    a.kt_lpt = plan->d_kt_lpt;
     a.fqtiles = plan->d_fqtiles;
     a.fentries = plan->d_fentries;
     a.fkt_off = plan->d_fkt_off;
@@ -546,7 +540,7 @@ int thd_cp_attn_bwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     a.status = plan->d_status;
     const int64_t nkt = plan->n_qtiles();
     if (nkt == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)nkt, plan->fkt_seg.back(), num_sms_current(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, plan->fkt_seg.back(), num_sms_current(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

@@ -7,29 +7,22 @@
 // dV summed over every rank that read a key (what a reduce-scatter of the gathered
 // gradients delivers; on one GPU the shared buffer already holds the sum).
 //
-// Three kernels, none with atomics:
-//   bwd_prep   Delta_i = sum_d dO_id O_id per (row, head).
-//   dkdv       one CTA per (key tile, key/value head g), groups outermost and key
-//              tiles longest-first within a group; it walks every query tile the
-//              plan's key-tile transpose lists (outer, latest query position first)
-//              and every query head of g's group (inner).  Key rows on TMEM lanes:
-//                a  S^T  = K Q^T   -> TMEM A       b  dP^T = V dO^T -> TMEM B
-//                phase 1: P^T = exp(S^T - lse) -> bf16 over S^T (A)
-//                phase 2: dS^T = P^T (dP^T - Delta) -> bf16 over dP^T (B)
-//                c  dV += P^T dO   (A operand from TMEM A)
-//                d  dK += dS^T Q   (A operand from TMEM B)
-//              issued as c(i), a(i+1), d(i), b(i+1): the exponentials of step i+1
-//              run while d(i) and b(i+1) are on the tensor pipe.  dK, dV stay in
-//              TMEM for the whole walk and are written once.
-//   dq         one CTA per (query tile, query head), like the forward: per listed
-//              entry S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - Delta) as bf16
-//              over S, dQ += dS K with the A operand from TMEM; written once.
-// Recomputing S and dP in the dq kernel costs 3/5 more tensor work than a single
-// kernel that reduces partial dQ tiles into global memory, but the reductions of
-// the single kernel move 64 KB per (query tile, key tile, head) through L2 and cap
-// at the L2's reduction bandwidth once dQ outgrows L2.
-#include <cstdlib>
-
+// Two kernels:
+//   bwd_prep   Delta_i = sum_d dO_id O_id per (row, head); zeroes dQ, dK and dV.
+//   bwd_fused  key-major: one CTA per (list segment of a key tile, key/value head g)
+//              walks the (query tile, query head) steps the plan lists for it and
+//              computes every gradient once per step (no tile is recomputed):
+//                a  S^T  = K Q^T   -> TMEM X       b  dP^T = V dO^T -> TMEM Y
+//                P^T = exp(S^T - lse), bf16 over S^T; dS^T = P^T (dP^T - Delta), bf16
+//                into shared memory (128-byte swizzled)
+//                c  dV += P^T dO   d  dK += dS^T Q   (accumulated in TMEM)
+//                e  Y = dS K: the key tile's share of the step's dQ, added into the
+//                   fp32 dQ by TMA tensor reductions (whole 128-byte row segments)
+//              dK, dV of the segment are added the same way at the end.
+// A query tile's dQ gathers shares from every key tile that sees it, so dQ is summed
+// at L2 (fp32 additions); an earlier design without additions, a key-major dK/dV
+// kernel plus a query-major dQ kernel, recomputed S and dP for dQ (3/5 more tensor
+// work) and was 10-25% slower end to end.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -107,569 +100,20 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) delta[(int64_t)(w % hq) * T + w / hq] = s;
-        // the fused kernel accumulates dQ, dK and dV with reductions: they start at zero
-        if (dq_zero) *reinterpret_cast<float4*>(dq_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (dk_zero && w < kv_rows) {
+        // dQ, dK and dV are accumulated with reductions: they start at zero
+        *reinterpret_cast<float4*>(dq_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (w < kv_rows) {
             *reinterpret_cast<float4*>(dk_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4*>(dv_zero + w * kD + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
 }
 
-// ================================================================ dK / dV
-struct DkdvLayout {
-    static constexpr int kQStages = 3, kDOStages = 2;
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = kOffK + kTile;
-    static constexpr int kOffQ = kOffV + kTile;
-    static constexpr int kOffDO = kOffQ + kQStages * kTile;
-    static constexpr int kOffStat = kOffDO + kDOStages * kTile;  // per dO stage: lse2[128], delta[128]
-    static constexpr int kOffBar = kOffStat + kDOStages * 256 * 4;
-    static constexpr int kBytes = kOffBar + 256;
-    static_assert(kBytes <= 232448, "shared memory budget");
-};
-
-// S^T and dP^T completions are signalled on three staged barriers each (step it uses
-// copy it % 3): besides the compute warpgroups, the producer recycles its Q and dO
-// stages on them, so the issuer commits twice per step, and with three copies the
-// phase the producer awaits is never ambiguous.
-struct DkdvBars {
-    uint64_t kv_full, q_full[3], do_full[2], stat_free[2], s_full[3], dp_full[3], p_ready, ds_ready, acc_done;
-    uint32_t tmem_base;
-    int abort;
-};
-
-__global__ void __launch_bounds__(kThreads, 1)
-dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
-    using L = DkdvLayout;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t base = smem_u32(smem_raw);
-    DkdvBars* bars = reinterpret_cast<DkdvBars*>(smem_raw + L::kOffBar);
-    float* s_stat = reinterpret_cast<float*>(smem_raw + L::kOffStat);
-    const uint32_t sK = base + L::kOffK, sV = base + L::kOffV, sQ = base + L::kOffQ, sDO = base + L::kOffDO;
-    volatile int* abort = &bars->abort;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int group = a.hq / a.hkv;
-    // Groups outermost: the CTAs resident together serve one KV group, so they read
-    // the same query heads, and (their lists being prefixes of one order) the same
-    // query tiles at about the same time; the tiles are mostly L2 hits after the first.
-    const int n_kt = (int)(gridDim.x / (unsigned)a.hkv);
-    const int kt = a.kt_lpt[blockIdx.x % n_kt];
-    const int g = blockIdx.x / n_kt;
-    const int* KT = a.qtiles + (size_t)kt * 12;  // key tiles are the plan's row tiles
-    const int k0 = KT[2], kn = KT[3];
-    const int l0 = a.kt_off[kt], llen = a.kt_off[kt + 1] - l0;
-    const int n_it = group * llen;
-
-    if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bars->kv_full), 1);
-        for (int s = 0; s < 3; ++s) {
-            mbar_init(smem_u32(&bars->q_full[s]), 1);
-            mbar_init(smem_u32(&bars->s_full[s]), 1);
-            mbar_init(smem_u32(&bars->dp_full[s]), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->do_full[s]), 1 + 32);        // expect_tx + the warp's lse/Delta stores
-            mbar_init(smem_u32(&bars->stat_free[s]), kCompute);    // Delta of the stage read by every thread
-        }
-        mbar_init(smem_u32(&bars->p_ready), kCompute);
-        mbar_init(smem_u32(&bars->ds_ready), kCompute);
-        mbar_init(smem_u32(&bars->acc_done), 1);
-        // the swizzled layout needs the 1024-byte alignment the declaration asks for
-        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
-        if (base & 1023u) atomicCAS(a.status, 0, 99);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (bars->abort) return;  // misaligned, or an earlier CTA timed out: do nothing
-    if (warp == 1) {
-        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = bars->tmem_base;
-    const uint32_t tA = tmem, tB = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
-
-    if (warp == 0) {
-        // ---------------------------------------------------- producer warp
-        const float log2e = 1.4426950408889634f;
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            tma_prefetch_desc(&tmDO);
-            const uint32_t kvf = smem_u32(&bars->kv_full);
-            mbar_arrive_expect_tx(kvf, 2 * kTile);
-            for (int c = 0; c < 2; ++c) {
-                tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
-                tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
-            }
-        }
-        StepMeta cur = load_meta(a.kt_list, a.qtiles, a.entries, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + 1);
-        for (int it = 0; it < n_it; ++it) {
-            const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
-            if (hh == 0 && it > 0) {
-                cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + pos + 1);
-            }
-            const int h = g * group + hh;
-            const int row0 = cur.row0;
-            float lv[4], dv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t row = (int64_t)row0 + lane + 32 * u;
-                lv[u] = row < a.T ? __ldg(a.lse + (int64_t)h * a.T + row) * log2e : 0.f;
-                dv[u] = row < a.T ? __ldg(a.delta + (int64_t)h * a.T + row) : 0.f;
-            }
-            const int qs = it % 3, ds = it & 1;
-            // Q(it) refills the stage d(it-3) read; b(it-2) is issued after d(it-3).
-            // dO(it) refills the stage c(it-2) read; a(it-1) is issued after c(it-2).
-            // The next use of either staged barrier needs a tile not loaded yet.
-            if (it >= 3) mbar_wait(smem_u32(&bars->dp_full[(it - 2) % 3]), ((it - 2) / 3) & 1, abort, a.status, 21);
-            if (lane == 0) {
-                const uint32_t f = smem_u32(&bars->q_full[qs]);
-                mbar_arrive_expect_tx(f, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + qs * kTile + c * kBox, f, c * 64, h, row0);
-            }
-            if (it >= 2) {
-                mbar_wait(smem_u32(&bars->s_full[(it - 1) % 3]), ((it - 1) / 3) & 1, abort, a.status, 22);
-                mbar_wait(smem_u32(&bars->stat_free[ds]), ((it >> 1) - 1) & 1, abort, a.status, 22);
-            }
-            const uint32_t f = smem_u32(&bars->do_full[ds]);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(f, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + ds * kTile + c * kBox, f, c * 64, h, row0);
-            }
-            float* stat = s_stat + ds * 256;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                stat[lane + 32 * u] = lv[u];
-                stat[128 + lane + 32 * u] = dv[u];
-            }
-            mbar_arrive(f);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // A, B K-major
-            constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);   // A TMEM, B MN-major
-            // descriptors: constant high word, low words advanced by a constant per K-step
-            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
-            const uint32_t klo = smem_desc_lo(sK, 16), vlo = smem_desc_lo(sV, 16);
-            auto issue_s = [&](int it) {  // a: S^T = K Q^T -> A
-                const int qs = it % 3;
-                mbar_wait(smem_u32(&bars->q_full[qs]), (it / 3) & 1, abort, a.status, 23);
-                tc_fence_after();
-                const uint32_t qlo = smem_desc_lo(sQ + qs * kTile, 16);
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-                    mma_ss(tA, smem_desc_of(klo + off, dhi), smem_desc_of(qlo + off, dhi), idKK, kk > 0);
-                }
-                mma_commit(smem_u32(&bars->s_full[it % 3]));
-            };
-            auto issue_dp = [&](int it) {  // b: dP^T = V dO^T -> B
-                const int ds = it & 1;
-                mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 24);
-                tc_fence_after();
-                const uint32_t dlo = smem_desc_lo(sDO + ds * kTile, 16);
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-                    mma_ss(tB, smem_desc_of(vlo + off, dhi), smem_desc_of(dlo + off, dhi), idKK, kk > 0);
-                }
-                mma_commit(smem_u32(&bars->dp_full[it % 3]));
-            };
-            mbar_wait(smem_u32(&bars->kv_full), 0, abort, a.status, 25);
-            tc_fence_after();
-            issue_s(0);
-            issue_dp(0);
-            for (int it = 0; it < n_it; ++it) {
-                const int qs = it % 3, ds = it & 1;
-                // c: dV += P^T dO, once P^T is in A
-                mbar_wait(smem_u32(&bars->p_ready), it & 1, abort, a.status, 26);
-                tc_fence_after();
-                const uint32_t dlo = smem_desc_lo(sDO + ds * kTile, kBox);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDV, tA + kk * 8, smem_desc_of(dlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
-                // a of the next step: A is rewritten only after c has read it (issue order)
-                if (it + 1 < n_it) issue_s(it + 1);
-                // d: dK += dS^T Q, once dS^T is in B
-                mbar_wait(smem_u32(&bars->ds_ready), it & 1, abort, a.status, 27);
-                tc_fence_after();
-                const uint32_t qlo = smem_desc_lo(sQ + qs * kTile, kBox);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tDK, tB + kk * 8, smem_desc_of(qlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
-                // b of the next step: B is rewritten only after d has read it (issue order)
-                if (it + 1 < n_it) issue_dp(it + 1);
-            }
-            mma_commit(smem_u32(&bars->acc_done));
-        }
-    } else {
-        // ---------------------------------------------------- compute warpgroups
-        const int ct = threadIdx.x - 64;         // 0..255
-        const int hf = ct >> 7;                  // column half
-        const int wq = warp & 3;
-        const int r = wq * 32 + lane;            // TMEM lane = key row
-        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-        const float sl2 = a.scale_log2;
-        const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
-        StepMeta cur = load_meta(a.kt_list, a.qtiles, a.entries, l0), nxt = cur;
-        if (llen > 1) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + 1);
-        for (int it = 0; it < n_it; ++it) {
-            const int ds = it & 1;
-            const int pos = it / group, hh = it - pos * group;
-            if (hh == 0 && it > 0) {
-                cur = nxt;
-                if (pos + 1 < llen) nxt = load_meta(a.kt_list, a.qtiles, a.entries, l0 + pos + 1);
-            }
-            const int m = cur.m, qpos0 = cur.qpos0, qbrk = cur.qbrk, qjump = cur.qjump;
-            // visible query columns of this key row: a suffix [lo, hi) of the tile
-            int lo = 0, hi = m;
-            if (r >= cur.nvalid) hi = 0;
-            else if (cur.cls != 2) {
-                const int n1 = min(qbrk, m);
-                if (kpos_r <= qpos0) lo = 0;
-                else if (kpos_r - qpos0 < n1) lo = kpos_r - qpos0;
-                else {
-                    const int p1 = qpos0 + qbrk + qjump;   // position of row qbrk
-                    lo = (kpos_r <= p1) ? n1 : min(m, n1 + (kpos_r - p1));
-                }
-            }
-            const float* stat = s_stat + ds * 256;
-
-            // ---- phase 1: P^T = exp(S^T - lse) on this thread's 64 query columns
-            mbar_wait(smem_u32(&bars->do_full[ds]), (it >> 1) & 1, abort, a.status, 28);  // lse/Delta staged
-            mbar_wait(smem_u32(&bars->s_full[it % 3]), (it / 3) & 1, abort, a.status, 29);
-            tc_fence_after();
-            float p[64];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t sv[32];
-                const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(tA + lane_addr + c0, sv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int t = 0; t < 32; t += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(stat + c0 + t);
-                    const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = c0 + t + u;
-                        const float e = ex2(fmaf(__uint_as_float(sv[t + u]), sl2, -lq[u]));
-                        p[ch * 32 + t + u] = (i >= lo && i < hi) ? e : 0.f;
-                    }
-                }
-            }
-            named_bar_sync(1, kCompute);  // all S^T reads of A are done before P^T overwrites it
-            {
-                uint32_t pk[32];
-#pragma unroll
-                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(p[2 * t], p[2 * t + 1]);
-                tmem_st32(tA + lane_addr + hf * 32, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->p_ready));
-
-            // ---- phase 2: dS^T = P^T (dP^T - Delta)
-            mbar_wait(smem_u32(&bars->dp_full[it % 3]), (it / 3) & 1, abort, a.status, 30);
-            tc_fence_after();
-            uint32_t dk[32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t dpv[32];
-                const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(tB + lane_addr + c0, dpv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int t = 0; t < 32; t += 4) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(stat + 128 + c0 + t);
-                    const float dq4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float dsv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) dsv[u] = p[ch * 32 + t + u] * (__uint_as_float(dpv[t + u]) - dq4[u]);
-                    dk[ch * 16 + t / 2] = pack_bf16x2(dsv[0], dsv[1]);
-                    dk[ch * 16 + t / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-                }
-            }
-            mbar_arrive(smem_u32(&bars->stat_free[ds]));  // Delta of this stage read
-            named_bar_sync(1, kCompute);  // all dP^T reads of B are done before dS^T overwrites it
-            tmem_st32(tB + lane_addr + hf * 32, dk);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->ds_ready));
-        }
-        // ---------------------------------------------------- dK, dV epilogue
-        mbar_wait(smem_u32(&bars->acc_done), 0, abort, a.status, 31);
-        tc_fence_after();
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-            const uint32_t src = which == 0 ? tDK : tDV;
-            float* out = which == 0 ? a.dk : a.dv;
-            const float mul = which == 0 ? a.scale : 1.f;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t v[32];
-                const int c0 = hf * 64 + ch * 32;
-                tmem_ld32(src + lane_addr + c0, v);
-                tmem_wait_ld();
-                if (r < kn) {
-                    float4* dst = reinterpret_cast<float4*>(out + ((int64_t)(k0 + r) * a.hkv + g) * kD + c0);
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        dst[t] = make_float4(__uint_as_float(v[4 * t]) * mul, __uint_as_float(v[4 * t + 1]) * mul,
-                                             __uint_as_float(v[4 * t + 2]) * mul, __uint_as_float(v[4 * t + 3]) * mul);
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-}
-
-// ================================================================ dQ
-struct DqLayout {
-    static constexpr int kKStages = 3, kVStages = 2;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffDO = kOffQ + kTile;
-    static constexpr int kOffK = kOffDO + kTile;
-    static constexpr int kOffV = kOffK + kKStages * kTile;
-    static constexpr int kOffBar = kOffV + kVStages * kTile;
-    static constexpr int kBytes = kOffBar + 256;
-    static_assert(kBytes <= 232448, "shared memory budget");
-};
-
-// The producer recycles K and V stages on the (double-buffered) S signal: S_{j-1} is
-// issued after dQ_{j-3} (last reader of K_j's stage) and dP_{j-2} (last reader of
-// V_j's), so the issuer commits twice per step.
-struct DqBars {
-    uint64_t qdo_full, k_full[3], v_full[2], s_full[2], dp_full, dp_free, ds_ready, dq_done;
-    uint32_t tmem_base;
-    int abort;
-};
-
-__global__ void __launch_bounds__(kThreads, 1)
-dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, BwdArgs a) {
-    using L = DqLayout;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t base = smem_u32(smem_raw);
-    DqBars* bars = reinterpret_cast<DqBars*>(smem_raw + L::kOffBar);
-    const uint32_t sQ = base + L::kOffQ, sDO = base + L::kOffDO, sK = base + L::kOffK, sV = base + L::kOffV;
-    volatile int* abort = &bars->abort;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int item = blockIdx.x;
-    const int qt = a.lpt[item / a.hq];
-    const int h = item % a.hq;
-    const int g = h / (a.hq / a.hkv);
-    const int* QT = a.qtiles + (size_t)qt * 12;
-    const int row0 = QT[2], m = QT[3], qpos0 = QT[4], qbrk = QT[5], qjump = QT[6];
-    const int nk = QT[8], e0 = QT[9];
-    const int* E = a.entries + (size_t)e0 * 8;
-
-    if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bars->qdo_full), 1);
-        for (int s = 0; s < 3; ++s) mbar_init(smem_u32(&bars->k_full[s]), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars->v_full[s]), 1);
-            mbar_init(smem_u32(&bars->s_full[s]), 1);
-        }
-        mbar_init(smem_u32(&bars->dp_full), 1);
-        mbar_init(smem_u32(&bars->dp_free), kCompute);
-        mbar_init(smem_u32(&bars->ds_ready), kCompute);
-        mbar_init(smem_u32(&bars->dq_done), 1);
-        bars->abort = (base & 1023u) ? 1 : *reinterpret_cast<volatile int*>(a.status);
-        if (base & 1023u) atomicCAS(a.status, 0, 99);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (bars->abort) return;
-    if (warp == 1) {
-        tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = bars->tmem_base;
-    const uint32_t tS = tmem, tDP = tmem + 256, tDQ = tmem + 384;   // S0 [0,128), S1 [128,256)
-
-    if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ TMA producer
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            tma_prefetch_desc(&tmDO);
-            const uint32_t f = smem_u32(&bars->qdo_full);
-            mbar_arrive_expect_tx(f, 2 * kTile);
-            for (int c = 0; c < 2; ++c) {
-                tma_load_3d(&tmQ, sQ + c * kBox, f, c * 64, h, row0);
-                tma_load_3d(&tmDO, sDO + c * kBox, f, c * 64, h, row0);
-            }
-            int k0_next = nk > 0 ? __ldg(E) : 0;
-            for (int j = 0; j < nk; ++j) {
-                const int k0 = k0_next;
-                if (j + 1 < nk) k0_next = __ldg(E + (j + 1) * 8);
-                const int ks = j % 3, vs = j & 1;
-                // S_{j-1} retired: dQ_{j-3} and dP_{j-2} are done.  The next use of that S
-                // barrier needs K_{j+1}, not loaded yet.
-                if (j >= 2) mbar_wait(smem_u32(&bars->s_full[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort, a.status, 41);
-                const uint32_t kf = smem_u32(&bars->k_full[ks]);
-                mbar_arrive_expect_tx(kf, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmK, sK + ks * kTile + c * kBox, kf, c * 64, g, k0);
-                const uint32_t vf = smem_u32(&bars->v_full[vs]);
-                mbar_arrive_expect_tx(vf, kTile);
-                for (int c = 0; c < 2; ++c) tma_load_3d(&tmV, sV + vs * kTile + c * kBox, vf, c * 64, g, k0);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idTM = idesc_bf16_f32(128, 128, false, true);
-            // descriptors: constant high word, low words advanced by a constant per K-step
-            constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
-            const uint32_t qlo = smem_desc_lo(sQ, 16), dolo = smem_desc_lo(sDO, 16);
-            mbar_wait(smem_u32(&bars->qdo_full), 0, abort, a.status, 43);
-            tc_fence_after();
-            for (int j = 0; j <= nk; ++j) {
-                if (j < nk) {
-                    const int ks = j % 3, vs = j & 1, b = j & 1;
-                    // S_j = Q K_j^T into S buffer b (it held dS_{j-2}, consumed by dQ_{j-2} issued earlier)
-                    mbar_wait(smem_u32(&bars->k_full[ks]), (j / 3) & 1, abort, a.status, 44);
-                    tc_fence_after();
-                    const uint32_t klo = smem_desc_lo(sK + ks * kTile, 16);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-                        mma_ss(tS + b * 128, smem_desc_of(qlo + off, dhi), smem_desc_of(klo + off, dhi), idKK, kk > 0);
-                    }
-                    mma_commit(smem_u32(&bars->s_full[b]));
-                    // dP_j = dO V_j^T, once dP_{j-1} has been read
-                    mbar_wait(smem_u32(&bars->v_full[vs]), (j >> 1) & 1, abort, a.status, 45);
-                    if (j >= 1) mbar_wait(smem_u32(&bars->dp_free), (j - 1) & 1, abort, a.status, 46);
-                    tc_fence_after();
-                    const uint32_t vlo = smem_desc_lo(sV + vs * kTile, 16);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-                        mma_ss(tDP, smem_desc_of(dolo + off, dhi), smem_desc_of(vlo + off, dhi), idKK, kk > 0);
-                    }
-                    mma_commit(smem_u32(&bars->dp_full));
-                }
-                if (j >= 1) {
-                    // dQ += dS_{j-1} K_{j-1}, dS from TMEM
-                    const int jj = j - 1, ks = jj % 3, b = jj & 1;
-                    mbar_wait(smem_u32(&bars->ds_ready), jj & 1, abort, a.status, 47);
-                    tc_fence_after();
-                    const uint32_t kmlo = smem_desc_lo(sK + ks * kTile, kBox);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tDQ, tS + b * 128 + kk * 8, smem_desc_of(kmlo + kk * (2048 >> 4), dhi), idTM,
-                               (jj > 0 || kk > 0));
-                }
-            }
-            mma_commit(smem_u32(&bars->dq_done));
-        }
-    } else {
-        // ---------------------------------------------------- compute warpgroups
-        const int ct = threadIdx.x - 64;
-        const int hf = ct >> 7;                  // key-column half
-        const int wq = warp & 3;
-        const int r = wq * 32 + lane;            // TMEM lane = query row
-        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-        const float sl2 = a.scale_log2;
-        const int qpos = qpos0 + r + (r >= qbrk ? qjump : 0);
-        const int64_t grow = (int64_t)row0 + r;
-        const float lse2 = grow < a.T ? __ldg(a.lse + (int64_t)h * a.T + grow) * 1.4426950408889634f : 0.f;
-        const float delta = grow < a.T ? __ldg(a.delta + (int64_t)h * a.T + grow) : 0.f;
-        int4 e_lo = make_int4(0, 0, 0, 0), e_hi = make_int4(0, 0, 0, 0);
-        if (nk > 0) {
-            e_lo = __ldg(reinterpret_cast<const int4*>(E));
-            e_hi = __ldg(reinterpret_cast<const int4*>(E) + 1);
-        }
-        for (int j = 0; j < nk; ++j) {
-            const int b = j & 1;
-            const int4 c_lo = e_lo, c_hi = e_hi;
-            if (j + 1 < nk) {
-                e_lo = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
-                e_hi = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8) + 1);
-            }
-            // record: k0, nvalid, kpos0, kbrk | kjump, cls, ktile, key_rank
-            int cnt = (r < m) ? c_lo.y : 0;
-            if (r < m && c_hi.y != 2) cnt = visible_keys(qpos, c_lo.y, c_lo.z, c_lo.w, c_hi.x);
-            mbar_wait(smem_u32(&bars->s_full[b]), (j >> 1) & 1, abort, a.status, 48);
-            mbar_wait(smem_u32(&bars->dp_full), j & 1, abort, a.status, 49);
-            tc_fence_after();
-            uint32_t sv[2][32], dpv[2][32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                tmem_ld32(tS + b * 128 + lane_addr + hf * 64 + ch * 32, sv[ch]);
-                tmem_ld32(tDP + lane_addr + hf * 64 + ch * 32, dpv[ch]);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->dp_free));
-            uint32_t pk[32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                for (int t = 0; t < 32; t += 2) {
-                    const int i = hf * 64 + ch * 32 + t;
-                    float p0 = ex2(fmaf(__uint_as_float(sv[ch][t]), sl2, -lse2));
-                    float p1 = ex2(fmaf(__uint_as_float(sv[ch][t + 1]), sl2, -lse2));
-                    p0 = i < cnt ? p0 : 0.f;
-                    p1 = i + 1 < cnt ? p1 : 0.f;
-                    pk[ch * 16 + t / 2] = pack_bf16x2(p0 * (__uint_as_float(dpv[ch][t]) - delta),
-                                                      p1 * (__uint_as_float(dpv[ch][t + 1]) - delta));
-                }
-            named_bar_sync(1, kCompute);  // all S reads of buffer b are done before dS overwrites it
-            tmem_st32(tS + b * 128 + lane_addr + hf * 32, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->ds_ready));
-        }
-        // ---------------------------------------------------- dQ epilogue
-        mbar_wait(smem_u32(&bars->dq_done), 0, abort, a.status, 50);
-        tc_fence_after();
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-            uint32_t v[32];
-            const int c0 = hf * 64 + ch * 32;
-            tmem_ld32(tDQ + lane_addr + c0, v);
-            tmem_wait_ld();
-            if (r < m) {
-                float4* dst = reinterpret_cast<float4*>(a.dq_acc + ((int64_t)(row0 + r) * a.hq + h) * kD + c0);
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    dst[t] = make_float4(__uint_as_float(v[4 * t]) * a.scale, __uint_as_float(v[4 * t + 1]) * a.scale,
-                                         __uint_as_float(v[4 * t + 2]) * a.scale,
-                                         __uint_as_float(v[4 * t + 3]) * a.scale);
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-}
-
-
 // ================================================================ fused dK / dV / dQ
-// One CTA per (key tile, key/value head g), walked like dkdv_kernel, and in the same
-// walk dQ: per step (query tile, query head)
+// One CTA per (list segment of a key tile, key/value head g).  Warp 0 loads K and V
+// once and then, per step (query tile outer, the group's query heads inner), Q, dO and
+// the rows' lse / Delta; warp 1 owns TMEM and issues every MMA; warps 2-9 are two
+// compute warpgroups (key row on the TMEM lane, 64 query columns per thread).  Per step:
 //   a  S^T  = K Q^T          -> TMEM X        b  dP^T = V dO^T -> TMEM Y
 //   P^T = exp(S^T - lse) as bf16 over S^T (X); dS^T = P^T (dP^T - Delta) as bf16 into
 //   shared memory (128-byte swizzled, the layout of a [key][query] tile)
@@ -677,7 +121,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 //   d  dK += dS^T Q   (A = dS^T from shared memory, K-major)
 //   e  Y   = dS K     (A = dS from the same bytes read MN-major: this CTA's share of
 //                      the query tile's dQ), drained by the compute warps and added
-//                      into the fp32 dQ with vector reductions at L2
+//                      into the fp32 dQ at L2
 // issued as c(i), a(i+1), d(i), e(i), b(i+1).  No tile is computed twice.
 struct FusedLayout {
     static constexpr int kOffK = 0;
@@ -1156,41 +600,23 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }  // namespace
 
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int n_items_per_group, int num_sms,
+                     const CUtensorMap& dout, const BwdArgs& a, int n_items_per_group, int num_sms,
                      cudaStream_t stream) {
     if (dqk != kD || dv != kD) return -2;
-    static const bool fused = [] {
-        const char* e = getenv("THD_BWD_SPLIT");
-        return !(e && e[0] == '1');
-    }();
-    const unsigned kv_grid = (unsigned)((int64_t)n_tiles * a.hkv);
-    if (fused) {
-        static std::atomic<uint64_t> fused_configured{0};
-        if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, fused_configured)) return -1;
-        CUtensorMap mdq, mdk, mdv, mqg, mkg, mvg, mdog;
-        if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&mdk, a.dk, a.T, a.hkv, kD) ||
-            !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&mqg, a.q, a.T * a.hq, kD) ||
-            !make_map_bf16_rows(&mkg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&mvg, a.v, a.T * a.hkv, kD) ||
-            !make_map_bf16_rows(&mdog, a.dout, a.T * a.hq, kD))
-            return -1;
-        bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.dk, a.dv, a.T * a.hkv,
-                                                         a.T * a.hq, a.hq, a.T);
-        if (cudaGetLastError() != cudaSuccess) return -1;
-        const unsigned items = (unsigned)((int64_t)n_items_per_group * a.hkv);
-        bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, mqg, mkg,
-                                                                           mvg, mdog, a);
-        return cudaGetLastError() == cudaSuccess ? 0 : -1;
-    }
-    static std::atomic<uint64_t> dkdv_configured{0}, dq_configured{0};
-    if (!ensure_dynamic_smem(dkdv_kernel, DkdvLayout::kBytes, dkdv_configured) ||
-        !ensure_dynamic_smem(dq_kernel, DqLayout::kBytes, dq_configured))
+    static std::atomic<uint64_t> configured{0};
+    if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, configured)) return -1;
+    CUtensorMap mdq, mdk, mdv, mqg, mkg, mvg, mdog;
+    if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&mdk, a.dk, a.T, a.hkv, kD) ||
+        !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&mqg, a.q, a.T * a.hq, kD) ||
+        !make_map_bf16_rows(&mkg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&mvg, a.v, a.T * a.hkv, kD) ||
+        !make_map_bf16_rows(&mdog, a.dout, a.T * a.hq, kD))
         return -1;
-    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, nullptr, nullptr, nullptr, 0,
+    bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.dk, a.dv, a.T * a.hkv,
                                                      a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
-    dkdv_kernel<<<kv_grid, kThreads, DkdvLayout::kBytes, stream>>>(q, k, v, dout, a);
-    if (cudaGetLastError() != cudaSuccess) return -1;
-    dq_kernel<<<(unsigned)((int64_t)n_tiles * a.hq), kThreads, DqLayout::kBytes, stream>>>(q, k, v, dout, a);
+    const unsigned items = (unsigned)((int64_t)n_items_per_group * a.hkv);
+    bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, mqg, mkg, mvg,
+                                                                       mdog, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -81,12 +81,6 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
         !thd::make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !thd::make_map_bf16(&mdo, do_rm, plan->T, hq, dv))
         return THD_ERR_CUDA;
     thd::BwdArgs a;
-    a.qtiles = plan->d_qtiles;
-    a.entries = plan->d_entries;
-    a.lpt = plan->d_lpt;
-    a.kt_off = plan->d_kt_off;
-    a.kt_list = plan->d_kt_list;
-    a.kt_lpt = plan->d_kt_lpt;
     a.fqtiles = plan->d_fqtiles;
     a.fentries = plan->d_fentries;
     a.fkt_off = plan->d_fkt_off;
@@ -112,7 +106,7 @@ extern "C" int thd_cp_attn_bwd_noalloc(thd_cp_plan_t plan, const void* q_rm, con
     a.scale_log2 = scale * 1.4426950408889634f;
     a.status = plan->d_status;
     if (plan->n_qtiles() == 0) return THD_OK;
-    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, (int)plan->n_qtiles(), plan->fkt_seg.back(), sm_count(),
+    return thd::launch_bwd_sm100(dqk, dv, mq, mk, mv, mdo, a, plan->fkt_seg.back(), sm_count(),
                                  static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;

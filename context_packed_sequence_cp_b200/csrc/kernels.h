@@ -82,12 +82,6 @@ int launch_fwd_f32(int dqk, int dv, const FwdF32Args& a, int n_items, cudaStream
 
 // ---- backward, bf16 on tcgen05 ---------------------------------------------------
 struct BwdArgs {
-    const int32_t* qtiles;
-    const int32_t* entries;
-    const int32_t* lpt;
-    const int32_t* kt_off;
-    const int32_t* kt_list;
-    const int32_t* kt_lpt;
     // the fused kernel walks the forward tables (rank-major and position tiles) and their
     // key-tile transpose; position rows are found through rm_of_global
     const int32_t* fqtiles;
@@ -114,10 +108,10 @@ struct BwdArgs {
     float scale_log2;
     int* status;
 };
-// n_tiles: key tiles; n_items_per_group: backward work items per key/value head
-// (kt_seg[n_kseg], the list segments of every key tile).
+// n_items_per_group: backward work items per key/value head (fkt_seg[n_fkseg], the list
+// segments of every key tile of the forward tables).
 int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& dout, const BwdArgs& a, int n_tiles, int n_items_per_group, int num_sms,
+                     const CUtensorMap& dout, const BwdArgs& a, int n_items_per_group, int num_sms,
                      cudaStream_t stream);
 
 // ---- rotary position embedding (half-split), per-document positions ---------------
