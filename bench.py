@@ -532,6 +532,30 @@ def run_native(args):
     rope_bytes = 2 * T * w.hq * w.dqk * 2 + T * (w.dqk // 2) * 8 * 2 + 4 * T
     del q_rope, rope_ws
 
+    # ------------------------------------------------ K/V all-gather fused into the forward's loads
+    # thd_cp_attn_fwd_fused_gather reads K/V from the packed tensors; compared with the
+    # step's K/V gather + forward on the same inputs (launches timed back to back).
+    def fg_time(fn, reps=3):
+        for _ in range(2):
+            fn()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        for _ in range(reps):
+            fn()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        return a_.elapsed_time(b_) / reps
+
+    def split():
+        thd.thd_kv_gather(plan, k, v, k_rm=k_rm, v_rm=v_rm)
+        thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm, out=o_rm, lse=lse_rm)
+
+    fused_ms = fg_time(lambda: thd.thd_cp_attn_fwd_fused_gather(plan, q_rm, k, v, out=o_rm, lse=lse_rm))
+    split_ms = fg_time(split)
+    fused_gather = {"ms": fused_ms, "tflops": fwd_fl / (fused_ms / 1e3) / 1e12, "gather_plus_fwd_ms": split_ms,
+                    "note": "thd_cp_attn_fwd_fused_gather (K/V read from the packed tensors) against "
+                            "thd_kv_gather(K, V) + thd_cp_attn_fwd, outside the timed step"}
+
     # ------------------------------------------------ re-plan for a new layout, other workloads
     peaks, peak_src = load_peaks()
     replan = measure_replan(thd, syn, plan, dev, stream, args.seed, w)
@@ -577,6 +601,7 @@ def run_native(args):
                  "note": "thd_cp_plan + thd_cp_plan_upload, once per layout (cached), outside the timed step",
                  "replan": replan},
         "workloads": workloads,
+        "fused_gather": fused_gather,
         "gather": {"ms": gather_ms, "gbs": gather_gbs, "frac_of_hbm": gather_gbs / hbm, "bytes": gather_bytes,
                    "hbm_peak_gbs": hbm, "peak_source": peak_src},
         "e2e": e2e,

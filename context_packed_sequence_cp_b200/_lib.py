@@ -37,6 +37,8 @@ SIGNATURES = {
     "thd_kv_gather": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _P]),
     "thd_rows_to_global": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
     "thd_cp_attn_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _F, _I32, _P]),
+    "thd_cp_attn_fwd_fused_gather": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _F, _I32,
+                                                    _P]),
     "thd_cu_seqlens_from_eod": (ctypes.c_int, [_P, ctypes.c_int64, _I32, _P, _I32, _P]),
     "thd_position_ids": (ctypes.c_int, [_P, _I32, _P]),
     "thd_rope_workspace": (ctypes.c_int, [ctypes.c_int64, _I32, _P]),

@@ -312,6 +312,28 @@ def thd_cp_attn_fwd(plan: Plan, q_rm: torch.Tensor, k_rm: torch.Tensor, v_rm: to
     return out, lse
 
 
+def thd_cp_attn_fwd_fused_gather(plan: Plan, q_rm: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
+                                 scale: float | None = None, out: torch.Tensor | None = None,
+                                 lse: torch.Tensor | None = None, stream=None):
+    """thd_cp_attn_fwd with K/V given in packed (global) order: the K/V all-gather is fused
+    into the attention's loads.  q_rm is rank-major; returns (o_rm, lse_rm [hq, T])."""
+    fn = "thd_cp_attn_fwd_fused_gather"
+    dev = _ready(fn, plan)
+    hq, hkv, dqk, dv = _qkv(fn, plan, dev, q_rm, k, v)
+    T = plan.T
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    dt = _dtype_code(fn, q_rm)
+    out = torch.empty((T, hq, dv), dtype=q_rm.dtype, device=q_rm.device) if out is None else out
+    lse = torch.empty((hq, T), dtype=torch.float32, device=q_rm.device) if lse is None else lse
+    _want(fn, "out", out, dev, (T, hq, dv), q_rm.dtype)
+    _want(fn, "lse", lse, dev, (hq, T), torch.float32)
+    check(fn, lib().thd_cp_attn_fwd_fused_gather(
+        plan.handle, _ptr(q_rm), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), hq, hkv, dqk, dv, float(scale), dt,
+        _stream(stream)))
+    return out, lse
+
+
 def thd_cp_attn_fwd_mla(plan: Plan, q_rm: torch.Tensor, k_nope_rm: torch.Tensor, k_rope_rm: torch.Tensor,
                         v_rm: torch.Tensor, *, scale: float | None = None, out: torch.Tensor | None = None,
                         lse: torch.Tensor | None = None, stream=None):

@@ -408,6 +408,7 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
     a.entries = plan->d_fentries;
     a.lpt = plan->d_flpt;
     a.rm_of_global = plan->d_rm_of_global;
+    a.kv_global = 0;
     a.o = static_cast<__nv_bfloat16*>(o_rm);
     a.lse = lse_rm;
     a.hq = hq;
@@ -448,6 +449,7 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
         a.entries = plan->d_fentries;
         a.lpt = plan->d_flpt;
         a.rm_of_global = plan->d_rm_of_global;
+        a.kv_global = 0;
         a.o = static_cast<__nv_bfloat16*>(o_rm);
         a.lse = lse_rm;
         a.hq = hq;
@@ -478,6 +480,42 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
         return thd::launch_fwd_f32(dqk, dv, a, (int)items, s) ? THD_ERR_CUDA : THD_OK;
     }
     return THD_ERR_UNSUPPORTED;
+}
+
+int thd_cp_attn_fwd_fused_gather(thd_cp_plan_t plan, const void* q_rm, const void* k, const void* v, void* o_rm,
+                                 float* lse_rm, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, float scale,
+                                 int32_t dtype, void* stream) {
+    int rc = ready(plan);
+    if (rc) return rc;
+    if (!q_rm || !k || !v || !o_rm || !lse_rm || !std::isfinite(scale) || !(scale > 0.f)) return THD_ERR_INVALID_ARG;
+    if ((rc = check_heads(hq, hkv))) return rc;
+    if (dtype != THD_DTYPE_BF16 || !((dqk == 128 && dv == 128) || (dqk == 192 && dv == 128))) return THD_ERR_UNSUPPORTED;
+    if (!aligned16(q_rm) || !aligned16(k) || !aligned16(v) || !aligned16(o_rm) || !aligned16(lse_rm))
+        return THD_ERR_MISALIGNED;
+    const int64_t items = plan->n_fqtiles() * (int64_t)hq;
+    if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
+    CUtensorMap mq, mk, mv, mqg, mkg, mvg;
+    if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k, plan->T, hkv, dqk) ||
+        !make_map_bf16(&mv, v, plan->T, hkv, dv) || !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, dqk) ||
+        !make_map_bf16_rows(&mkg, k, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v, plan->T * hkv, dv))
+        return THD_ERR_CUDA;
+    thd::FwdArgs a;
+    a.qtiles = plan->d_fqtiles;
+    a.entries = plan->d_fentries;
+    a.lpt = plan->d_flpt;
+    a.rm_of_global = plan->d_rm_of_global;
+    a.kv_global = 1;
+    a.o = static_cast<__nv_bfloat16*>(o_rm);
+    a.lse = lse_rm;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.T = plan->T;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.status = plan->d_status;
+    if (items == 0) return THD_OK;
+    return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)items, static_cast<cudaStream_t>(stream))
+               ? THD_ERR_CUDA
+               : THD_OK;
 }
 
 int thd_cp_attn_bwd_workspace(thd_cp_plan_t plan, int32_t hq, int32_t hkv, int32_t dqk, int32_t dv, int32_t dtype,

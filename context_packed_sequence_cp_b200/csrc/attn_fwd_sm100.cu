@@ -194,17 +194,35 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tma_prefetch_desc(&tmV);
         }
         const int ns = is_k ? NK : NV;
-        int4 e_next = nk > 0 ? __ldg(reinterpret_cast<const int4*>(E)) : make_int4(0, 0, 0, 0);
+        // Where entry j's K/V rows come from: box_row >= 0 is the first row of one box of
+        // 128 consecutive rows; otherwise the 4 rows of this lane are gathered (rr).
+        //   rank-major K/V (kv_global == 0): rank-major tiles are boxes at k0; position
+        //   tiles gather rank-major rows through rm_of_global.
+        //   packed K/V (kv_global != 0; the gather of K/V fused into the loads): a run of
+        //   consecutive positions is a box at kpos0; a rank-major run with a seam gathers
+        //   its positions.
+        auto locate = [&](int j, int (&rr)[4]) {
+            const int4 lo = __ldg(reinterpret_cast<const int4*>(E + j * 8));   // k0, nvalid, kpos0, kbrk
+            if (!a.kv_global) {
+                if (lo.x < 0) gather_index(lo.z, lo.y, rr);
+                return lo.x;
+            }
+            const int kjump = __ldg(E + j * 8 + 4);
+            if (lo.w >= lo.y || kjump == 0) return lo.z;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = min(lane * 4 + i, lo.y - 1);
+                rr[i] = lo.z + t + (t >= lo.w ? kjump : 0);
+            }
+            return -1;
+        };
         int rr_next[4] = {0, 0, 0, 0};
-        if (nk > 0 && e_next.x < 0) gather_index(e_next.z, e_next.y, rr_next);
+        int box_next = nk > 0 ? locate(0, rr_next) : 0;
         for (int j = 0; j < nk; ++j) {
             const int st = j % ns;
-            const int4 e = e_next;   // k0, nvalid, kpos0, -
+            const int box_row = box_next;
             int rr[4] = {rr_next[0], rr_next[1], rr_next[2], rr_next[3]};
-            if (j + 1 < nk) {
-                e_next = __ldg(reinterpret_cast<const int4*>(E + (j + 1) * 8));
-                if (e_next.x < 0) gather_index(e_next.z, e_next.y, rr_next);
-            }
+            if (j + 1 < nk) box_next = locate(j + 1, rr_next);
             // A stage is refilled once the MMA that read it has retired: K_{j-NK} is
             // read by S_{j-NK} (signalled on s_full), V_{j-NV} by PV_{j-NV} (o_done).
             // NK, NV <= kSBuf, so the next use of either barrier needs the tile
@@ -215,13 +233,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const uint32_t kf = smem_u32(&bars->k_full[st]);
                 if (lane == 0) mbar_arrive_expect_tx(kf, L::kKBytes);
                 __syncwarp();
-                if (e.x >= 0) {
+                if (box_row >= 0) {
                     if (lane == 0)
                         for (int c = 0; c < DQK / 64; ++c) {
                             if (SHARED_ROPE && c == 2)
-                                tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, e.x);
+                                tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, box_row);
                             else
-                                tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, e.x);
+                                tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, g, box_row);
                         }
                 } else if (SHARED_ROPE) {   // per-head part, then the shared rope key (one row per token)
                     gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, a.hkv, g, 0, 2);
@@ -235,10 +253,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const uint32_t vf = smem_u32(&bars->v_full[st]);
                 if (lane == 0) mbar_arrive_expect_tx(vf, L::kVBytes);
                 __syncwarp();
-                if (e.x >= 0) {
+                if (box_row >= 0) {
                     if (lane == 0)
                         for (int c = 0; c < DV / 64; ++c)
-                            tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, e.x);
+                            tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, g, box_row);
                 } else {
                     gather_rows(&tmVg, sV + st * L::kVBytes, vf, rr, a.hkv, g, 0, DV / 64);
                 }

@@ -46,6 +46,7 @@ struct FwdArgs {
     const int32_t* entries;
     const int32_t* lpt;
     const int32_t* rm_of_global;  // rows of position tiles (row0 / k0 < 0)
+    int32_t kv_global;            // K/V given in packed (global) order: rows are positions
     __nv_bfloat16* o;
     float* lse;
     int32_t hq, hkv;

@@ -306,6 +306,27 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
                     int32_t dv, float scale, int32_t dtype, void* stream);
 
 /*
+ * thd_cp_attn_fwd_fused_gather -- thd_cp_attn_fwd with the K/V all-gather fused into
+ * the attention's loads ([WHAT] KV all-gather with direct rank-major indexing: the
+ * key/value rows a rank-major tile needs are fetched straight from the packed
+ * tensors by position, so the rank-major K/V copy of thd_kv_gather is not needed).
+ * Same attention, outputs and errors as thd_cp_attn_fwd; the query side stays
+ * rank-major (a rank's own rows).
+ *   q_rm [T, hq, dqk] rank-major; k [T, hkv, dqk], v [T, hkv, dv] in packed (global)
+ *   order; o_rm [T, hq, dv] rank-major; lse_rm fp32 [hq, T].
+ *   A key tile whose positions are consecutive (every tile of a document with chunks of
+ *   128 or more rows, and every position tile) is one TMA box at its first position; a
+ *   rank-major tile holding the seam between a rank's two chunks gathers its rows
+ *   (TMA tile::gather4).  The loaded tiles are the rows thd_cp_attn_fwd reads from the
+ *   rank-major copy, in the same order, so the outputs are bit-identical to it.
+ *   Supported: THD_DTYPE_BF16 with (dqk, dv) in {(128,128), (192,128)}.
+ */
+int thd_cp_attn_fwd_fused_gather(thd_cp_plan_t plan, const void* q_rm, const void* k,
+                                 const void* v, void* o_rm, float* lse_rm, int32_t hq,
+                                 int32_t hkv, int32_t dqk, int32_t dv, float scale,
+                                 int32_t dtype, void* stream);
+
+/*
  * thd_cp_attn_fwd_mla -- thd_cp_attn_fwd for multi-head latent attention whose keys
  * are given in compact form: a per-head part and one rotary-position ("rope") key
  * per token shared by every head.  [WHAT] lists MLA among the head layouts the path

@@ -140,3 +140,29 @@ def test_fwd_bf16_position_tiles_around_the_chunk_threshold(cp):
     want_o, want_l = A.attention_fwd(q, k, v, cu, 1 / math.sqrt(128))
     assert_bf16_close(o, want_o, "O")
     assert np.abs(lse - want_l).max() <= LSE_MAX
+
+
+@pytest.mark.parametrize("cp,chunks,heads", [(4, [1, 17, 64, 127, 128, 129, 300, 3], (8, 2)),
+                                              (16, [160, 32, 200], (8, 1)), (1, [900, 5], (4, 4))])
+def test_fwd_fused_gather_is_bit_identical(cp, chunks, heads):
+    """K/V read straight from the packed tensors (the all-gather fused into the loads):
+    boxes for runs of consecutive positions, gathers for runs with a seam; the outputs
+    equal thd_cp_attn_fwd's on the rank-major copy bit for bit, and the oracle's."""
+    import context_packed_sequence_cp_b200 as thd
+    hq, hkv = heads
+    cu = syn.cu_seqlens_of([2 * cp * c for c in chunks])
+    q, k, v = syn.make_tensors(int(cu[-1]), hq, hkv, 128, 128, torch.bfloat16, seed=60 + cp, device="cuda")
+    plan = thd.Plan(cu, cp).upload()
+    q_rm = thd.thd_kv_gather(plan, q)
+    k_rm, v_rm = thd.thd_kv_gather(plan, k, v)
+    o_ref, l_ref = thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm)
+    o_fg, l_fg = thd.thd_cp_attn_fwd_fused_gather(plan, q_rm, k, v)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    assert torch.equal(o_fg, o_ref) and torch.equal(l_fg, l_ref)
+    if int(cu[-1]) <= 8192:
+        q_idx = plan.export()["q_idx"]
+        from tests.gpu_util import unpermute_rows
+        o = unpermute_rows(o_fg.float().cpu().numpy(), q_idx)
+        want_o, _ = A.attention_fwd(q.cpu(), k.cpu(), v.cpu(), cu, 1 / math.sqrt(128))
+        assert_bf16_close(o, want_o, "O")
