@@ -290,7 +290,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 lv[u] = rs[u] >= 0 ? __ldg(a.lse + (int64_t)h * a.T + rs[u]) * log2e : 0.f;
-                dv[u] = rs[u] >= 0 ? __ldg(a.delta + (int64_t)h * a.T + rs[u]) : 0.f;
+                dv[u] = rs[u] >= 0 ? __ldg(a.delta + (int64_t)h * a.T + rs[u]) * a.scale : 0.f;
             }
             const int st = it & 1;
             // dO(it) refills the stage c(it-2) read: c(it-2) is issued before a(it-1).
@@ -407,6 +407,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int r = wq * 32 + lane;            // TMEM lane: key row (X, Y as S^T / dP^T), query row (Y as dQ)
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sl2 = a.scale_log2;
+        const float sc = a.scale;
         const int kpos_r = KT[4] + r + (r >= KT[5] ? KT[6] : 0);
         // this thread's 128-byte row of dS^T: box hf, row r, 16-byte chunks swizzled by r % 8
         const uint32_t ds_row = sDS + hf * kBox + r * 128;
@@ -421,14 +422,11 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // into global memory with a TMA tensor reduction (whole 128-byte row segments).  A
         // warp whose rows run past the tile's valid rows adds those with vector reductions.
         const uint32_t warp_stage = sDS + hf * kBox + wq * 32 * 128;
-        auto stage = [&](const uint32_t (&v)[32], float mul) {  // chunks swizzled by lane % 8
+        auto stage = [&](const uint32_t (&v)[32]) {  // chunks swizzled by lane % 8
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-                st_shared_v4(warp_stage + lane * 128 + ((c ^ (lane & 7)) << 4),
-                             __float_as_uint(__uint_as_float(v[4 * c]) * mul),
-                             __float_as_uint(__uint_as_float(v[4 * c + 1]) * mul),
-                             __float_as_uint(__uint_as_float(v[4 * c + 2]) * mul),
-                             __float_as_uint(__uint_as_float(v[4 * c + 3]) * mul));
+                st_shared_v4(warp_stage + lane * 128 + ((c ^ (lane & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2],
+                             v[4 * c + 3]);
         };
         // The staging rows are rewritten only after stage_free(): a box handed to the TMA unit
         // is waited for (read out of shared memory) there, as late as possible.
@@ -472,14 +470,14 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             uint32_t v[32];
             tmem_ld32(tY + lane_addr + hf * 64, v);
             tmem_wait_ld();
-            stage(v, a.scale);
+            stage(v);
             tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
             reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             stage_free();
-            stage(v, a.scale);
+            stage(v);
             reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
         };
         for (int it = 0; it < n_it; ++it) {
@@ -559,8 +557,9 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     for (int u = 0; u < 4; ++u) {
                         const int t = j * 8 + 2 * u;
                         const float2 d2 = *reinterpret_cast<const float2*>(stat + 128 + c0 + t);
-                        w4[u] = pack_bf16x2(p[ch * 32 + t] * (__uint_as_float(dpv[t]) - d2.x),
-                                            p[ch * 32 + t + 1] * (__uint_as_float(dpv[t + 1]) - d2.y));
+                        // scale folded in: scale * dS = P (scale * dP - scale * Delta)
+                        w4[u] = pack_bf16x2(p[ch * 32 + t] * fmaf(__uint_as_float(dpv[t]), sc, -d2.x),
+                                            p[ch * 32 + t + 1] * fmaf(__uint_as_float(dpv[t + 1]), sc, -d2.y));
                     }
                     const int chunk = ch * 4 + j;
                     if (ch == 0 && j == 0) stage_free();   // the drain's last box has been read
@@ -586,7 +585,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tmem_ld32(src + lane_addr + hf * 64 + ch * 32, v);
                 tmem_wait_ld();
                 stage_free();
-                stage(v, which == 0 ? a.scale : 1.f);
+                stage(v);
                 reduce(which == 0 ? &tmDK : &tmDV, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kpos0, kn, hf * 64 + ch * 32);
             }
         }
