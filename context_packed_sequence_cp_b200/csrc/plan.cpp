@@ -240,47 +240,74 @@ int thd_build_plan(const int32_t* cu, int32_t n_docs, int32_t cp, thd_cp_plan_s*
         // s + v*BM .. (read in place from the rank-major buffers through rm_of_global),
         // key tiles 0 .. u listed for query tile u, the last one the diagonal.  Rank-major
         // records are marked by row0 / k0 >= 0; position records carry -1 there.
-        // An entry's key tile (field 6) is the forward tile that holds its keys.
-        p->fqtiles.clear();
-        p->fentries.clear();
+        // An entry's key tile (field 6) is the forward tile that holds its keys.  Sizes are
+        // counted first, so that both tables are allocated once and filled in place.
         std::vector<int32_t> f_of_tile(n_tiles, -1);  // forward index of a rank-major tile
-        int32_t nf_rm = 0;
-        for (int64_t t = 0; t < n_tiles; ++t)
-            if (lay.chunk(p->qtiles[(size_t)t * THD_QTILE_FIELDS + 1]) >= BM) f_of_tile[t] = nf_rm++;
+        int64_t nf = 0, nfe = 0;
         for (int64_t t = 0; t < n_tiles; ++t) {
             const int32_t* q = &p->qtiles[(size_t)t * THD_QTILE_FIELDS];
+            if (lay.chunk(q[1]) < BM) continue;
+            f_of_tile[t] = (int32_t)nf++;
+            nfe += q[8];
+        }
+        for (int d = 0; d < n_docs; ++d)
+            if (lay.chunk(d) < BM) {
+                const int64_t n = ceil_div(L[d], BM);
+                nf += n;
+                nfe += n * (n + 1) / 2;
+            }
+        if (nfe > std::numeric_limits<int32_t>::max() / 2) return THD_ERR_INVALID_ARG;
+        p->fqtiles.assign((size_t)nf * THD_QTILE_FIELDS, 0);
+        p->fentries.assign((size_t)nfe * THD_ENTRY_FIELDS, 0);
+        int32_t* fq = p->fqtiles.data();
+        int32_t* fe = p->fentries.data();
+        int64_t ft = 0, fn = 0;  // tiles and entries written
+        for (int64_t t = 0; t < n_tiles; ++t) {
             if (f_of_tile[t] < 0) continue;
-            const int32_t off = (int32_t)(p->fentries.size() / THD_ENTRY_FIELDS);
-            p->fqtiles.insert(p->fqtiles.end(), q, q + THD_QTILE_FIELDS);
-            p->fqtiles[p->fqtiles.size() - THD_QTILE_FIELDS + 9] = off;
-            p->fentries.insert(p->fentries.end(), p->entries.begin() + (size_t)q[9] * THD_ENTRY_FIELDS,
-                               p->entries.begin() + (size_t)(q[9] + q[8]) * THD_ENTRY_FIELDS);
-            for (int64_t e = off; e < (int64_t)off + q[8]; ++e) {
-                int32_t& kt = p->fentries[(size_t)e * THD_ENTRY_FIELDS + 6];
-                kt = f_of_tile[kt];
+            const int32_t* q = &p->qtiles[(size_t)t * THD_QTILE_FIELDS];
+            std::copy(q, q + THD_QTILE_FIELDS, fq + ft * THD_QTILE_FIELDS);
+            fq[ft * THD_QTILE_FIELDS + 9] = (int32_t)fn;
+            ++ft;
+            const int32_t* src = &p->entries[(size_t)q[9] * THD_ENTRY_FIELDS];
+            for (int32_t k = 0; k < q[8]; ++k, ++fn) {
+                int32_t* e = fe + fn * THD_ENTRY_FIELDS;
+                std::copy(src + (size_t)k * THD_ENTRY_FIELDS, src + (size_t)(k + 1) * THD_ENTRY_FIELDS, e);
+                e[6] = f_of_tile[e[6]];
             }
         }
         for (int d = 0; d < n_docs; ++d) {
             if (lay.chunk(d) >= BM) continue;
             const int64_t n = ceil_div(L[d], BM);
-            const int32_t first_tile = (int32_t)(p->fqtiles.size() / THD_QTILE_FIELDS);  // position tile 0 of d
-            for (int64_t u = 0; u < n; ++u) {
+            const int32_t first_tile = (int32_t)ft;  // position tile 0 of d
+            for (int64_t u = 0; u < n; ++u, ++ft) {
                 const int64_t p0 = s[d] + u * BM, m = std::min<int64_t>(BM, L[d] - u * BM), qmax = p0 + m - 1;
-                const int32_t rec[THD_QTILE_FIELDS] = {-1, d, -1, (int32_t)m, (int32_t)p0, (int32_t)m, 0, (int32_t)qmax,
-                                                       (int32_t)(u + 1),
-                                                       (int32_t)(p->fentries.size() / THD_ENTRY_FIELDS),
-                                                       (int32_t)s[d], (int32_t)(s[d] + L[d])};
-                p->fqtiles.insert(p->fqtiles.end(), rec, rec + THD_QTILE_FIELDS);
-                for (int64_t v = 0; v <= u; ++v) {
+                int32_t* q = fq + ft * THD_QTILE_FIELDS;
+                q[0] = -1;
+                q[1] = d;
+                q[2] = -1;
+                q[3] = (int32_t)m;
+                q[4] = (int32_t)p0;
+                q[5] = (int32_t)m;
+                q[6] = 0;
+                q[7] = (int32_t)qmax;
+                q[8] = (int32_t)(u + 1);
+                q[9] = (int32_t)fn;
+                q[10] = (int32_t)s[d];
+                q[11] = (int32_t)(s[d] + L[d]);
+                for (int64_t v = 0; v <= u; ++v, ++fn) {
                     const int64_t kp0 = s[d] + v * BM, nv = std::min<int64_t>(BM, qmax - kp0 + 1);
-                    const int32_t cls = kp0 + nv - 1 <= p0 ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
-                    const int32_t e[THD_ENTRY_FIELDS] = {-1, (int32_t)nv, (int32_t)kp0, (int32_t)nv, 0, cls,
-                                                         first_tile + (int32_t)v, -1};
-                    p->fentries.insert(p->fentries.end(), e, e + THD_ENTRY_FIELDS);
+                    int32_t* e = fe + fn * THD_ENTRY_FIELDS;
+                    e[0] = -1;
+                    e[1] = (int32_t)nv;
+                    e[2] = (int32_t)kp0;
+                    e[3] = (int32_t)nv;
+                    e[4] = 0;
+                    e[5] = kp0 + nv - 1 <= p0 ? THD_CLS_UNMASKED : THD_CLS_PARTIAL;
+                    e[6] = first_tile + (int32_t)v;
+                    e[7] = -1;
                 }
             }
         }
-        const int64_t nf = (int64_t)p->fqtiles.size() / THD_QTILE_FIELDS;
         p->flpt.resize(nf);
         for (int64_t t = 0; t < nf; ++t) p->flpt[t] = (int32_t)t;
         std::stable_sort(p->flpt.begin(), p->flpt.end(), [&](int32_t a, int32_t b) {
