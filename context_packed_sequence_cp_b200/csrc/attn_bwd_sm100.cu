@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 //   P^T = exp(S^T - lse) as bf16 over S^T (X); dS^T = P^T (dP^T - Delta) as bf16 into
 //   shared memory (128-byte swizzled, the layout of a [key][query] tile)
 //   c  dV += P^T dO   (A from TMEM X)
-//   d  dK += dS^T Q   (A = dS^T from shared memory, K-major)
+//   d  dK += dS^T Q   (A = dS^T, also stored as bf16 over dP^T in TMEM Y)
 //   e  Y   = dS K     (A = dS from the same bytes read MN-major: this CTA's share of
 //                      the query tile's dQ), drained by the compute warps and added
 //                      into the fp32 dQ at L2
@@ -335,7 +335,6 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             constexpr uint32_t dhi = smem_desc_hi_sw128(1024);
             const uint32_t klo = smem_desc_lo(sK, 16), vlo = smem_desc_lo(sV, 16);
             const uint32_t kmlo = smem_desc_lo(sK, kBox);   // K as the MN-major B of e
-            const uint32_t dslo = smem_desc_lo(sDS, 16);    // dS^T, K-major A of d
             const uint32_t dsmlo = smem_desc_lo(sDS, kBox); // dS, MN-major A of e
             auto issue_a = [&](int it) {  // S^T = K Q^T -> X
                 const int st = it & 1;
@@ -382,9 +381,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const uint32_t qlo = smem_desc_lo(sQ + st * kTile, kBox);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
-                    mma_ss(tDK, smem_desc_of(dslo + off, dhi), smem_desc_of(qlo + kk * (2048 >> 4), dhi), idTM,
-                           (it > 0 || kk > 0));
+                    mma_ts(tDK, tY + kk * 8, smem_desc_of(qlo + kk * (2048 >> 4), dhi), idTM, (it > 0 || kk > 0));
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -544,6 +541,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             // ---- P2: dS^T = P^T (dP^T - Delta) -> shared memory
             mbar_wait(smem_u32(&bars->dp_full), it & 1, abort, a.status, 73);
             tc_fence_after();
+            uint32_t dsk[32];
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 uint32_t dpv[32];
@@ -561,11 +559,18 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         w4[u] = pack_bf16x2(p[ch * 32 + t] * fmaf(__uint_as_float(dpv[t]), sc, -d2.x),
                                             p[ch * 32 + t + 1] * fmaf(__uint_as_float(dpv[t + 1]), sc, -d2.y));
                     }
+                    dsk[ch * 16 + j * 4] = w4[0];
+                    dsk[ch * 16 + j * 4 + 1] = w4[1];
+                    dsk[ch * 16 + j * 4 + 2] = w4[2];
+                    dsk[ch * 16 + j * 4 + 3] = w4[3];
                     const int chunk = ch * 4 + j;
                     if (ch == 0 && j == 0) stage_free();   // the drain's last box has been read
                     st_shared_v4(ds_row + ((chunk ^ (r & 7)) << 4), w4[0], w4[1], w4[2], w4[3]);
                 }
             }
+            named_bar_sync(2 + wq, 64);  // both halves have read dP^T before dS^T overwrites it
+            tmem_st32(tY + lane_addr + hf * 32, dsk);
+            tmem_wait_st();
             mbar_arrive(smem_u32(&bars->stat_free[st]));  // lse and Delta of this stage read
             fence_proxy_async_smem();                      // dS^T visible to the tensor pipe
             tc_fence_before();
