@@ -382,6 +382,34 @@ int thd_rows_to_global(thd_cp_plan_t plan, const void* src_rm, void* dst, int64_
     return THD_OK;
 }
 
+namespace {
+// Persistent CTAs (each taking over the items of CTAs that have not started) pay off when
+// items are short: a CTA's fill and drain (Q load, first S, epilogue) is then a large share
+// of an item and overlaps with the neighbouring items.  With long items one CTA per item
+// measured as fast or faster, so the plan's mean key tiles per query tile decides.
+constexpr int64_t kPersistMaxMeanTiles = 64;
+
+// Arguments of the bf16 forward over the forward tables.
+thd::FwdArgs fwd_args(thd_plan* plan, void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, float scale,
+                      int32_t kv_global) {
+    thd::FwdArgs a;
+    a.qtiles = plan->d_fqtiles;
+    a.entries = plan->d_fentries;
+    a.lpt = plan->d_flpt;
+    a.rm_of_global = plan->d_rm_of_global;
+    a.kv_global = kv_global;
+    a.persistent = plan->n_fentries() < kPersistMaxMeanTiles * plan->n_fqtiles() ? 1 : 0;
+    a.o = static_cast<__nv_bfloat16*>(o_rm);
+    a.lse = lse_rm;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.T = plan->T;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.status = plan->d_status;
+    return a;
+}
+}  // namespace
+
 int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope_rm, const void* k_rope_rm,
                         const void* v_rm, void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, int32_t d_nope,
                         int32_t d_rope, int32_t dv, float scale, int32_t dtype, void* stream) {
@@ -403,19 +431,7 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
         !make_map_bf16_rows(&mkng, k_nope_rm, plan->T * hkv, d_nope) ||
         !make_map_bf16_rows(&mkrg, k_rope_rm, plan->T, d_rope) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
         return THD_ERR_CUDA;
-    thd::FwdArgs a;   // the forward tables, as thd_cp_attn_fwd
-    a.qtiles = plan->d_fqtiles;
-    a.entries = plan->d_fentries;
-    a.lpt = plan->d_flpt;
-    a.rm_of_global = plan->d_rm_of_global;
-    a.kv_global = 0;
-    a.o = static_cast<__nv_bfloat16*>(o_rm);
-    a.lse = lse_rm;
-    a.hq = hq;
-    a.hkv = hkv;
-    a.T = plan->T;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.status = plan->d_status;
+    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);  // the forward tables
     if (items == 0) return THD_OK;
     return thd::launch_fwd_mla_sm100(mq, mkn, mkr, mv, mqg, mkng, mkrg, mvg, a, (int)items,
                                      static_cast<cudaStream_t>(stream))
@@ -444,19 +460,7 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
             !make_map_bf16_rows(&mkg, k_rm, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
             return THD_ERR_CUDA;
         // the forward tables: rank-major tiles, position tiles for short-chunk documents
-        thd::FwdArgs a;
-        a.qtiles = plan->d_fqtiles;
-        a.entries = plan->d_fentries;
-        a.lpt = plan->d_flpt;
-        a.rm_of_global = plan->d_rm_of_global;
-        a.kv_global = 0;
-        a.o = static_cast<__nv_bfloat16*>(o_rm);
-        a.lse = lse_rm;
-        a.hq = hq;
-        a.hkv = hkv;
-        a.T = plan->T;
-        a.scale_log2 = scale * 1.4426950408889634f;
-        a.status = plan->d_status;
+        const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);
         const int64_t fitems = plan->n_fqtiles() * (int64_t)hq;
         if (fitems == 0) return THD_OK;
         return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)fitems, s) ? THD_ERR_CUDA : THD_OK;
@@ -499,19 +503,7 @@ int thd_cp_attn_fwd_fused_gather(thd_cp_plan_t plan, const void* q_rm, const voi
         !make_map_bf16(&mv, v, plan->T, hkv, dv) || !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, dqk) ||
         !make_map_bf16_rows(&mkg, k, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v, plan->T * hkv, dv))
         return THD_ERR_CUDA;
-    thd::FwdArgs a;
-    a.qtiles = plan->d_fqtiles;
-    a.entries = plan->d_fentries;
-    a.lpt = plan->d_flpt;
-    a.rm_of_global = plan->d_rm_of_global;
-    a.kv_global = 1;
-    a.o = static_cast<__nv_bfloat16*>(o_rm);
-    a.lse = lse_rm;
-    a.hq = hq;
-    a.hkv = hkv;
-    a.T = plan->T;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.status = plan->d_status;
+    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 1);
     if (items == 0) return THD_OK;
     return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)items, static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA

@@ -233,6 +233,34 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- cluster launch control
+// Asks the hardware to cancel the launch of a CTA of this grid (clusters of one CTA) that
+// has not started yet.  The 16-byte response lands at `resp` (shared memory, 16-byte
+// aligned) and completes 16 transaction bytes on `bar`.  Once a response has cancelled
+// nothing, the CTA makes no further request.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+            resp),
+        "r"(bar)
+        : "memory");
+}
+
+// blockIdx.x of the CTA that a response cancelled, or -1 when it cancelled none (every
+// CTA of the grid has started or been taken over).
+__device__ __forceinline__ int clc_cancelled_x(uint32_t resp) {
+    int x = -1;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+        "ld.shared.b128 r, [%1];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, r;\n\t}"
+        : "+r"(x)
+        : "r"(resp)
+        : "memory");
+    return x;
+}
+
 // Four fp32 additions to consecutive global addresses, performed at L2 (no result).
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
