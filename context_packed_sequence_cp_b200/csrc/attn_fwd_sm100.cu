@@ -135,6 +135,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmQg, const __grid_constant__ CUtensorMap tmKg,
            const __grid_constant__ CUtensorMap tmVg, const __grid_constant__ CUtensorMap tmKrg, FwdArgs a) {
     static_assert(!SHARED_ROPE || DQK == 192, "the shared rope key is the third 64-column box");
+    static_assert(DV == 128, "the epilogue stores 8 chunks of 8 columns per half row");
     using L = FwdLayout<DQK, DV>;
     constexpr int NK = L::NK, NV = L::NV;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -268,10 +269,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int ns = is_k ? NK : NV;
         uint32_t J = 0;  // tiles of the CTA's earlier items
         int kq = 0;      // the CTA's earlier items with tiles
+        FwdItem x = fwd_item(blockIdx.x, a);
         for (int it = blockIdx.x, r = 0; it >= 0; ++r) {
-            const FwdItem x = fwd_item(it, a);
             const int nk = x.q2.x;
             const int* E = a.entries + (size_t)x.q2.y * 8;
+            // The rows of the item's Q (a position tile) and of its first K/V tile are looked
+            // up before the waits for a free buffer, so that their loads overlap the wait.
+            int rq[4] = {0, 0, 0, 0};
+            if (is_k && nk > 0 && x.q0.z < 0) gather_index(x.q1.x, x.q0.w, rq);
+            int rr_next[4] = {0, 0, 0, 0};
+            int box_next = nk > 0 ? locate(E, 0, rr_next) : 0;
             if (is_k && nk > 0) {
                 // One Q buffer, refilled once every S of the previous item has retired
                 // (q_free, committed after that item's last S).  A second buffer measured no
@@ -284,13 +291,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     if (lane == 0)
                         for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, x.h, x.q0.z);
                 } else {
-                    int rq[4];
-                    gather_index(x.q1.x, x.q0.w, rq);
                     gather_rows(&tmQg, sQ, qf, rq, a.hq, x.h, 0, DQK / 64);
                 }
             }
-            int rr_next[4] = {0, 0, 0, 0};
-            int box_next = nk > 0 ? locate(E, 0, rr_next) : 0;
             for (int j = 0; j < nk; ++j) {
                 const uint32_t Jj = J + j;
                 const int st = Jj % ns;
@@ -342,6 +345,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             kq += nk > 0;
             it = take_next(r, true);
             if (PERSIST && is_k && lane == 0 && it >= 0) request(r + 1);
+            if (it >= 0) x = fwd_item(it, a);
         }
     } else if (warp == 1 || warp == kPvWarp) {
         // ---------------------------------------------------- MMA issuers
@@ -572,18 +576,44 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->o_free));  // the next item's first PV may overwrite O
+            // This thread's DV/2 = 64 output columns as bf16, in 16-byte chunks of 8 columns.
+            uint4 ch[8];
 #pragma unroll
-            for (int c = 0; c < DV / 64; ++c) {
-                uint32_t pk[16];
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t* s = o[q >> 2] + (q & 3) * 8;
+                ch[q] = make_uint4(pack_bf16x2(__uint_as_float(s[0]) * inv_l, __uint_as_float(s[1]) * inv_l),
+                                   pack_bf16x2(__uint_as_float(s[2]) * inv_l, __uint_as_float(s[3]) * inv_l),
+                                   pack_bf16x2(__uint_as_float(s[4]) * inv_l, __uint_as_float(s[5]) * inv_l),
+                                   pack_bf16x2(__uint_as_float(s[6]) * inv_l, __uint_as_float(s[7]) * inv_l));
+            }
+            // 8 x 8 transposes of the chunks within each group of 8 lanes (8 rows), by XOR
+            // shuffles: afterwards lane i of a group holds chunk i of each of the group's rows,
+            // so that one store instruction writes four whole 128-byte half rows instead of
+            // 32 scattered 16-byte pieces (rows are hq * DV * 2 bytes apart).
+            const int gi = lane & 7;
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    pk[t] = pack_bf16x2(__uint_as_float(o[c][2 * t]) * inv_l, __uint_as_float(o[c][2 * t + 1]) * inv_l);
-                if (row < m) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            for (int k = 4; k >= 1; k >>= 1) {
+                const bool up = (gi & k) != 0;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                for (int j = 0; j < 8; ++j) {
+                    if (j & k) continue;
+                    uint4 x = up ? ch[j] : ch[j | k];
+                    x.x = __shfl_xor_sync(0xffffffffu, x.x, k);
+                    x.y = __shfl_xor_sync(0xffffffffu, x.y, k);
+                    x.z = __shfl_xor_sync(0xffffffffu, x.z, k);
+                    x.w = __shfl_xor_sync(0xffffffffu, x.w, k);
+                    if (up)
+                        ch[j] = x;
+                    else
+                        ch[j | k] = x;
                 }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int src = (lane & ~7) + j;  // the lane of row 8 * group + j
+                const unsigned long long p =
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(orow), src);
+                if (wq * 32 + src < m) *(reinterpret_cast<uint4*>(p) + gi) = ch[j];
             }
             if (row < m && hf == 0)
                 a.lse[(size_t)h * a.T + orow_idx] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
