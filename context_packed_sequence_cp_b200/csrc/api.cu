@@ -151,12 +151,12 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)dim * 2, (cuuint64_t)heads * dim * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -173,6 +173,23 @@ bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int di
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The forward's maps of Q [T, hq, dqk], K [T, hkv, dk], V [T, hkv, dv] and the shared rope
+// key K_rope [T, 1, dr] (kr; nullptr: K again): 128-row boxes, 8-row boxes, row maps.
+bool make_fwd_maps(thd::FwdMaps* m, int64_t T, const void* q, int hq, int dqk, const void* k, int hkv, int dk,
+                   const void* v, int dv, const void* kr, int dr) {
+    if (!kr) {
+        kr = k;
+        dr = dk;
+    }
+    const int hr = kr == k ? hkv : 1;
+    return make_map_bf16(&m->q, q, T, hq, dqk) && make_map_bf16(&m->k, k, T, hkv, dk) &&
+           make_map_bf16(&m->v, v, T, hkv, dv) && make_map_bf16(&m->kr, kr, T, hr, dr) &&
+           make_map_bf16(&m->q8, q, T, hq, dqk, 8) && make_map_bf16(&m->k8, k, T, hkv, dk, 8) &&
+           make_map_bf16(&m->v8, v, T, hkv, dv, 8) && make_map_bf16(&m->kr8, kr, T, hr, dr, 8) &&
+           make_map_bf16_rows(&m->qg, q, T * hq, dqk) && make_map_bf16_rows(&m->kg, k, T * hkv, dk) &&
+           make_map_bf16_rows(&m->vg, v, T * hkv, dv) && make_map_bf16_rows(&m->krg, kr, T * hr, dr);
 }
 
 bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
@@ -424,17 +441,12 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
         return THD_ERR_MISALIGNED;
     const int64_t items = plan->n_fqtiles() * (int64_t)hq;
     if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
-    CUtensorMap mq, mkn, mkr, mv, mqg, mkng, mkrg, mvg;
-    if (!make_map_bf16(&mq, q_rm, plan->T, hq, d_nope + d_rope) || !make_map_bf16(&mkn, k_nope_rm, plan->T, hkv, d_nope) ||
-        !make_map_bf16(&mkr, k_rope_rm, plan->T, 1, d_rope) || !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) ||
-        !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, d_nope + d_rope) ||
-        !make_map_bf16_rows(&mkng, k_nope_rm, plan->T * hkv, d_nope) ||
-        !make_map_bf16_rows(&mkrg, k_rope_rm, plan->T, d_rope) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
+    thd::FwdMaps maps;
+    if (!make_fwd_maps(&maps, plan->T, q_rm, hq, d_nope + d_rope, k_nope_rm, hkv, d_nope, v_rm, dv, k_rope_rm, d_rope))
         return THD_ERR_CUDA;
     const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);  // the forward tables
     if (items == 0) return THD_OK;
-    return thd::launch_fwd_mla_sm100(mq, mkn, mkr, mv, mqg, mkng, mkrg, mvg, a, (int)items,
-                                     static_cast<cudaStream_t>(stream))
+    return thd::launch_fwd_mla_sm100(maps, a, (int)items, static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;
 }
@@ -454,16 +466,13 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == THD_DTYPE_BF16) {
         if (!((dqk == 128 && dv == 128) || (dqk == 192 && dv == 128))) return THD_ERR_UNSUPPORTED;
-        CUtensorMap mq, mk, mv, mqg, mkg, mvg;
-        if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k_rm, plan->T, hkv, dqk) ||
-            !make_map_bf16(&mv, v_rm, plan->T, hkv, dv) || !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, dqk) ||
-            !make_map_bf16_rows(&mkg, k_rm, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v_rm, plan->T * hkv, dv))
-            return THD_ERR_CUDA;
+        thd::FwdMaps maps;
+        if (!make_fwd_maps(&maps, plan->T, q_rm, hq, dqk, k_rm, hkv, dqk, v_rm, dv, nullptr, 0)) return THD_ERR_CUDA;
         // the forward tables: rank-major tiles, position tiles for short-chunk documents
         const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);
         const int64_t fitems = plan->n_fqtiles() * (int64_t)hq;
         if (fitems == 0) return THD_OK;
-        return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)fitems, s) ? THD_ERR_CUDA : THD_OK;
+        return thd::launch_fwd_sm100(dqk, dv, maps, a, (int)fitems, s) ? THD_ERR_CUDA : THD_OK;
     }
     if (dtype == THD_DTYPE_FP32) {
         if (!((dqk == 64 && dv == 64) || (dqk == 128 && dv == 128))) return THD_ERR_UNSUPPORTED;
@@ -498,14 +507,11 @@ int thd_cp_attn_fwd_fused_gather(thd_cp_plan_t plan, const void* q_rm, const voi
         return THD_ERR_MISALIGNED;
     const int64_t items = plan->n_fqtiles() * (int64_t)hq;
     if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
-    CUtensorMap mq, mk, mv, mqg, mkg, mvg;
-    if (!make_map_bf16(&mq, q_rm, plan->T, hq, dqk) || !make_map_bf16(&mk, k, plan->T, hkv, dqk) ||
-        !make_map_bf16(&mv, v, plan->T, hkv, dv) || !make_map_bf16_rows(&mqg, q_rm, plan->T * hq, dqk) ||
-        !make_map_bf16_rows(&mkg, k, plan->T * hkv, dqk) || !make_map_bf16_rows(&mvg, v, plan->T * hkv, dv))
-        return THD_ERR_CUDA;
+    thd::FwdMaps maps;
+    if (!make_fwd_maps(&maps, plan->T, q_rm, hq, dqk, k, hkv, dqk, v, dv, nullptr, 0)) return THD_ERR_CUDA;
     const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 1);
     if (items == 0) return THD_OK;
-    return thd::launch_fwd_sm100(dqk, dv, mq, mk, mv, mqg, mkg, mvg, a, (int)items, static_cast<cudaStream_t>(stream))
+    return thd::launch_fwd_sm100(dqk, dv, maps, a, (int)items, static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
                : THD_OK;
 }

@@ -126,14 +126,11 @@ __device__ __forceinline__ int visible_prefix(int qpos, int nvalid, int kpos0, i
 }
 
 // SHARED_ROPE (DQK = 192 only): keys come in the compact form of multi-head latent
-// attention, a per-head 128-wide part (tmK) and one 64-wide rope key per token shared
-// by every head (tmKr); the third 64-column box of each key tile is read from tmKr.
+// attention, a per-head 128-wide part (tm.k) and one 64-wide rope key per token shared
+// by every head (tm.kr); the third 64-column box of each key tile is read from tm.kr.
 template <int DQK, int DV, bool SHARED_ROPE, bool PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
-fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKr,
-           const __grid_constant__ CUtensorMap tmQg, const __grid_constant__ CUtensorMap tmKg,
-           const __grid_constant__ CUtensorMap tmVg, const __grid_constant__ CUtensorMap tmKrg, FwdArgs a) {
+fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
     static_assert(!SHARED_ROPE || DQK == 192, "the shared rope key is the third 64-column box");
     static_assert(DV == 128, "the epilogue stores 8 chunks of 8 columns per half row");
     using L = FwdLayout<DQK, DV>;
@@ -208,40 +205,59 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // A rank-major tile (row0 / k0 >= 0) is a box of 128 consecutive rank-major rows,
         // loaded by lane 0.  A position tile (row0 / k0 < 0; short-chunk documents) holds
         // positions pos0 .. pos0+n-1, read in place from the rank-major buffer through
-        // rm_of_global: every lane gathers 4 rows per 64-column box (tile::gather4), rows
-        // past n repeat row n-1 (they are masked).
+        // rm_of_global, in groups of 8 rows: lane l takes group l % 16 and the 64-column
+        // boxes l / 16, l / 16 + 2, ...  A group whose rows are 8 consecutive rows of the
+        // buffer (inside one chunk) is one 8-row box, landing at the group's 1024-byte offset
+        // so that the swizzled layout is the full box's; any other group (one that crosses a
+        // chunk boundary or the tile's end) is two 4-row gathers (tile::gather4).  Rows past
+        // n repeat row n-1 (they are masked).
         const bool is_k = warp == 0;
-        // this lane's 4 rank-major rows of a position tile (their indices are loaded one
-        // tile ahead, so that the load latency overlaps the wait for a free stage)
-        auto gather_index = [&](int pos0, int n, int (&rr)[4]) {
+        // this lane's group of 8 rows of a position tile (the indices are loaded one tile
+        // ahead, so that the load latency overlaps the wait for a free stage)
+        auto group_index = [&](int pos0, int n, int (&rr)[8]) {
+            const int g8 = (lane & 15) * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1));
+            for (int i = 0; i < 8; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(g8 + i, n - 1));
         };
-        // 64-column boxes c0 .. c1-1 of those rows, row (rm * heads + head) of the row map
-        auto gather_rows = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int heads,
-                               int head, int c0, int c1) {
-            for (int c = c0; c < c1; ++c)
-                tma_gather4(map, dst + c * L::kBox + lane * 512, bar, (c - c0) * 64, rr[0] * heads + head,
-                            rr[1] * heads + head, rr[2] * heads + head, rr[3] * heads + head);
+        // 64-column boxes c0 .. c1-1 of those rows; a row r of the buffer is (r, head) of the
+        // 3-D map box8 and row r * heads + head of the row map
+        auto load_groups = [&](const CUtensorMap* box8, const CUtensorMap* rows, uint32_t dst, uint32_t bar,
+                               const int (&rr)[8], int heads, int head, int c0, int c1) {
+            bool run = true;
+#pragma unroll
+            for (int i = 1; i < 8; ++i) run = run && rr[i] == rr[0] + i;
+            const uint32_t gdst = dst + (lane & 15) * 1024;
+            for (int c = c0 + (lane >> 4); c < c1; c += 2) {
+                const uint32_t d = gdst + c * L::kBox;
+                if (run) {
+                    tma_load_3d(box8, d, bar, (c - c0) * 64, head, rr[0]);
+                } else {
+                    tma_gather4(rows, d, bar, (c - c0) * 64, rr[0] * heads + head, rr[1] * heads + head,
+                                rr[2] * heads + head, rr[3] * heads + head);
+                    tma_gather4(rows, d + 512, bar, (c - c0) * 64, rr[4] * heads + head, rr[5] * heads + head,
+                                rr[6] * heads + head, rr[7] * heads + head);
+                }
+            }
         };
         // Where entry j's K/V rows come from: box_row >= 0 is the first row of one box of
-        // 128 consecutive rows; otherwise the 4 rows of this lane are gathered (rr).
+        // 128 consecutive rows; otherwise this lane's group of 8 rows (rr).
         //   rank-major K/V (kv_global == 0): rank-major tiles are boxes at k0; position
-        //   tiles gather rank-major rows through rm_of_global.
+        //   tiles take rank-major rows through rm_of_global.
         //   packed K/V (kv_global != 0; the gather of K/V fused into the loads): a run of
-        //   consecutive positions is a box at kpos0; a rank-major run with a seam gathers
-        //   its positions.
-        auto locate = [&](const int* E, int j, int (&rr)[4]) {
+        //   consecutive positions is a box at kpos0; a rank-major run with a seam takes its
+        //   positions.
+        auto locate = [&](const int* E, int j, int (&rr)[8]) {
             const int4 lo = __ldg(reinterpret_cast<const int4*>(E + j * 8));  // k0, nvalid, kpos0, kbrk
             if (!a.kv_global) {
-                if (lo.x < 0) gather_index(lo.z, lo.y, rr);
+                if (lo.x < 0) group_index(lo.z, lo.y, rr);
                 return lo.x;
             }
             const int kjump = __ldg(E + j * 8 + 4);
             if (lo.w >= lo.y || kjump == 0) return lo.z;
+            const int g8 = (lane & 15) * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = min(lane * 4 + i, lo.y - 1);
+            for (int i = 0; i < 8; ++i) {
+                const int t = min(g8 + i, lo.y - 1);
                 rr[i] = lo.z + t + (t >= lo.w ? kjump : 0);
             }
             return -1;
@@ -258,12 +274,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         };
         if (lane == 0) {
             if (is_k) {
-                tma_prefetch_desc(&tmQ);
-                tma_prefetch_desc(&tmK);
-                if (SHARED_ROPE) tma_prefetch_desc(&tmKr);
+                tma_prefetch_desc(&tm.q);
+                tma_prefetch_desc(&tm.k);
+                if (SHARED_ROPE) tma_prefetch_desc(&tm.kr);
                 if (PERSIST) request(0);
             } else {
-                tma_prefetch_desc(&tmV);
+                tma_prefetch_desc(&tm.v);
             }
         }
         const int ns = is_k ? NK : NV;
@@ -275,9 +291,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int* E = a.entries + (size_t)x.q2.y * 8;
             // The rows of the item's Q (a position tile) and of its first K/V tile are looked
             // up before the waits for a free buffer, so that their loads overlap the wait.
-            int rq[4] = {0, 0, 0, 0};
-            if (is_k && nk > 0 && x.q0.z < 0) gather_index(x.q1.x, x.q0.w, rq);
-            int rr_next[4] = {0, 0, 0, 0};
+            int rq[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (is_k && nk > 0 && x.q0.z < 0) group_index(x.q1.x, x.q0.w, rq);
+            int rr_next[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             int box_next = nk > 0 ? locate(E, 0, rr_next) : 0;
             if (is_k && nk > 0) {
                 // One Q buffer, refilled once every S of the previous item has retired
@@ -289,16 +305,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 __syncwarp();
                 if (x.q0.z >= 0) {
                     if (lane == 0)
-                        for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tmQ, sQ + c * L::kBox, qf, c * 64, x.h, x.q0.z);
+                        for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tm.q, sQ + c * L::kBox, qf, c * 64, x.h, x.q0.z);
                 } else {
-                    gather_rows(&tmQg, sQ, qf, rq, a.hq, x.h, 0, DQK / 64);
+                    load_groups(&tm.q8, &tm.qg, sQ, qf, rq, a.hq, x.h, 0, DQK / 64);
                 }
             }
             for (int j = 0; j < nk; ++j) {
                 const uint32_t Jj = J + j;
                 const int st = Jj % ns;
                 const int box_row = box_next;
-                int rr[4] = {rr_next[0], rr_next[1], rr_next[2], rr_next[3]};
+                int rr[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) rr[i] = rr_next[i];
                 if (j + 1 < nk) box_next = locate(E, j + 1, rr_next);
                 // A stage is refilled once the MMA that read it has retired: K_{J-NK} is
                 // read by S_{J-NK} (signalled on s_full), V_{J-NV} by PV_{J-NV} (o_done).
@@ -315,15 +333,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                         if (lane == 0)
                             for (int c = 0; c < DQK / 64; ++c) {
                                 if (SHARED_ROPE && c == 2)
-                                    tma_load_3d(&tmKr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, box_row);
+                                    tma_load_3d(&tm.kr, sK + st * L::kKBytes + c * L::kBox, kf, 0, 0, box_row);
                                 else
-                                    tma_load_3d(&tmK, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, x.g, box_row);
+                                    tma_load_3d(&tm.k, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, x.g, box_row);
                             }
                     } else if (SHARED_ROPE) {  // per-head part, then the shared rope key (one row per token)
-                        gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, 2);
-                        gather_rows(&tmKrg, sK + st * L::kKBytes, kf, rr, 1, 0, 2, 3);
+                        load_groups(&tm.k8, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, 2);
+                        load_groups(&tm.kr8, &tm.krg, sK + st * L::kKBytes, kf, rr, 1, 0, 2, 3);
                     } else {
-                        gather_rows(&tmKg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, DQK / 64);
+                        load_groups(&tm.k8, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, DQK / 64);
                     }
                 } else {
                     if (Jj >= NV)
@@ -335,9 +353,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     if (box_row >= 0) {
                         if (lane == 0)
                             for (int c = 0; c < DV / 64; ++c)
-                                tma_load_3d(&tmV, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, x.g, box_row);
+                                tma_load_3d(&tm.v, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, x.g, box_row);
                     } else {
-                        gather_rows(&tmVg, sV + st * L::kVBytes, vf, rr, a.hkv, x.g, 0, DV / 64);
+                        load_groups(&tm.v8, &tm.vg, sV + st * L::kVBytes, vf, rr, a.hkv, x.g, 0, DV / 64);
                     }
                 }
             }
@@ -626,40 +644,30 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 template <int DQK, int DV, bool SHARED_ROPE, bool PERSIST>
-int launch_as(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr,
-              const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const CUtensorMap& krg,
-              const FwdArgs& a, int n_items, cudaStream_t stream) {
+int launch_as(const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream) {
     using L = FwdLayout<DQK, DV>;
     static std::atomic<uint64_t> configured{0};
     if (!ensure_dynamic_smem(fwd_kernel<DQK, DV, SHARED_ROPE, PERSIST>, L::kDynSmem, configured)) return -1;
-    fwd_kernel<DQK, DV, SHARED_ROPE, PERSIST><<<n_items, kThreads, L::kDynSmem, stream>>>(q, k, v, kr, qg, kg, vg,
-                                                                                         krg, a);
+    fwd_kernel<DQK, DV, SHARED_ROPE, PERSIST><<<n_items, kThreads, L::kDynSmem, stream>>>(m, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <int DQK, int DV, bool SHARED_ROPE>
-int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kr,
-           const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const CUtensorMap& krg,
-           const FwdArgs& a, int n_items, cudaStream_t stream) {
-    return a.persistent ? launch_as<DQK, DV, SHARED_ROPE, true>(q, k, v, kr, qg, kg, vg, krg, a, n_items, stream)
-                        : launch_as<DQK, DV, SHARED_ROPE, false>(q, k, v, kr, qg, kg, vg, krg, a, n_items, stream);
+int launch(const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream) {
+    return a.persistent ? launch_as<DQK, DV, SHARED_ROPE, true>(m, a, n_items, stream)
+                        : launch_as<DQK, DV, SHARED_ROPE, false>(m, a, n_items, stream);
 }
 
 }  // namespace
 
-int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a,
-                     int n_items, cudaStream_t stream) {
-    if (dqk == 128 && dv == 128) return launch<128, 128, false>(q, k, v, k, qg, kg, vg, kg, a, n_items, stream);
-    if (dqk == 192 && dv == 128) return launch<192, 128, false>(q, k, v, k, qg, kg, vg, kg, a, n_items, stream);
+int launch_fwd_sm100(int dqk, int dv, const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream) {
+    if (dqk == 128 && dv == 128) return launch<128, 128, false>(m, a, n_items, stream);
+    if (dqk == 192 && dv == 128) return launch<192, 128, false>(m, a, n_items, stream);
     return -2;
 }
 
-int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
-                         const CUtensorMap& v, const CUtensorMap& qg, const CUtensorMap& k_nope_g,
-                         const CUtensorMap& k_rope_g, const CUtensorMap& vg, const FwdArgs& a, int n_items,
-                         cudaStream_t stream) {
-    return launch<192, 128, true>(q, k_nope, v, k_rope, qg, k_nope_g, vg, k_rope_g, a, n_items, stream);
+int launch_fwd_mla_sm100(const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream) {
+    return launch<192, 128, true>(m, a, n_items, stream);
 }
 
 }  // namespace thd

@@ -24,9 +24,9 @@ inline bool ensure_dynamic_smem(Kernel* fn, int bytes, std::atomic<uint64_t>& do
 }
 
 // [rows, heads, dim] bf16 tensor viewed as a 3-D TMA map with 64-column x 1-head x
-// 128-row boxes and 128-byte swizzle (the layout the tcgen05 descriptors expect).
+// box_rows-row boxes and 128-byte swizzle (the layout the tcgen05 descriptors expect).
 // False when the driver's encoder is unavailable or rejects the map.
-bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
+bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim, int box_rows = 128);
 // [rows, dim] bf16 tensor (a [T, heads, dim] tensor seen as T * heads rows) viewed as a
 // 2-D TMA map with 64-column x 1-row boxes and 128-byte swizzle, for tile::gather4 loads.
 bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int dim);
@@ -55,16 +55,20 @@ struct FwdArgs {
     float scale_log2;  // scale * log2(e)
     int* status;       // device word: nonzero once a bounded wait gave up
 };
-// qg, kg, vg: the same tensors as 2-D row maps (make_map_bf16_rows), read by position tiles.
-int launch_fwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                     const CUtensorMap& qg, const CUtensorMap& kg, const CUtensorMap& vg, const FwdArgs& a,
-                     int n_items, cudaStream_t stream);
-// Multi-head latent attention with a shared rope key: Q [T, hq, 192], K_nope [T, hkv, 128],
-// K_rope [T, 1, 64] (one per token, every head), V [T, hkv, 128].
-int launch_fwd_mla_sm100(const CUtensorMap& q, const CUtensorMap& k_nope, const CUtensorMap& k_rope,
-                         const CUtensorMap& v, const CUtensorMap& qg, const CUtensorMap& k_nope_g,
-                         const CUtensorMap& k_rope_g, const CUtensorMap& vg, const FwdArgs& a, int n_items,
-                         cudaStream_t stream);
+// Tensor maps of the bf16 forward, over Q [T, hq, dqk], K [T, hkv, dqk], V [T, hkv, dv]
+// (and K_rope [T, 1, 64] of the compact multi-head latent attention form, else K again):
+//   q, k, v, kr      3-D {dim, heads, rows} maps, boxes of 64 columns x 128 rows;
+//   q8, k8, v8, kr8  the same with boxes of 8 rows (runs inside position tiles);
+//   qg, kg, vg, krg  2-D {dim, rows * heads} row maps, boxes of one row (tile::gather4).
+struct FwdMaps {
+    CUtensorMap q, k, v, kr;
+    CUtensorMap q8, k8, v8, kr8;
+    CUtensorMap qg, kg, vg, krg;
+};
+int launch_fwd_sm100(int dqk, int dv, const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream);
+// Multi-head latent attention with a shared rope key: Q [T, hq, 192], K_nope [T, hkv, 128] (k),
+// K_rope [T, 1, 64] (kr, one per token, every head), V [T, hkv, 128].
+int launch_fwd_mla_sm100(const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream);
 
 // ---- forward, fp32 SIMT --------------------------------------------------------
 struct FwdF32Args {
