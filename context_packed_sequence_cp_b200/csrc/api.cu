@@ -176,7 +176,7 @@ bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int di
 }
 
 // The forward's maps of Q [T, hq, dqk], K [T, hkv, dk], V [T, hkv, dv] and the shared rope
-// key K_rope [T, 1, dr] (kr; nullptr: K again): 128-row boxes, 8-row boxes, row maps.
+// key K_rope [T, 1, dr] (kr; nullptr: K again): 128-row boxes, 8- to 64-row boxes, row maps.
 bool make_fwd_maps(thd::FwdMaps* m, int64_t T, const void* q, int hq, int dqk, const void* k, int hkv, int dk,
                    const void* v, int dv, const void* kr, int dr) {
     if (!kr) {
@@ -184,10 +184,12 @@ bool make_fwd_maps(thd::FwdMaps* m, int64_t T, const void* q, int hq, int dqk, c
         dr = dk;
     }
     const int hr = kr == k ? hkv : 1;
+    for (int s = 0; s < thd::kRunBoxes; ++s)
+        if (!make_map_bf16(&m->qs[s], q, T, hq, dqk, 8 << s) || !make_map_bf16(&m->ks[s], k, T, hkv, dk, 8 << s) ||
+            !make_map_bf16(&m->vs[s], v, T, hkv, dv, 8 << s) || !make_map_bf16(&m->krs[s], kr, T, hr, dr, 8 << s))
+            return false;
     return make_map_bf16(&m->q, q, T, hq, dqk) && make_map_bf16(&m->k, k, T, hkv, dk) &&
            make_map_bf16(&m->v, v, T, hkv, dv) && make_map_bf16(&m->kr, kr, T, hr, dr) &&
-           make_map_bf16(&m->q8, q, T, hq, dqk, 8) && make_map_bf16(&m->k8, k, T, hkv, dk, 8) &&
-           make_map_bf16(&m->v8, v, T, hkv, dv, 8) && make_map_bf16(&m->kr8, kr, T, hr, dr, 8) &&
            make_map_bf16_rows(&m->qg, q, T * hq, dqk) && make_map_bf16_rows(&m->kg, k, T * hkv, dk) &&
            make_map_bf16_rows(&m->vg, v, T * hkv, dv) && make_map_bf16_rows(&m->krg, kr, T * hr, dr);
 }

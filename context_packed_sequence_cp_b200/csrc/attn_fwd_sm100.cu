@@ -206,11 +206,13 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
         // loaded by lane 0.  A position tile (row0 / k0 < 0; short-chunk documents) holds
         // positions pos0 .. pos0+n-1, read in place from the rank-major buffer through
         // rm_of_global, in groups of 8 rows: lane l takes group l % 16 and the 64-column
-        // boxes l / 16, l / 16 + 2, ...  A group whose rows are 8 consecutive rows of the
-        // buffer (inside one chunk) is one 8-row box, landing at the group's 1024-byte offset
-        // so that the swizzled layout is the full box's; any other group (one that crosses a
-        // chunk boundary or the tile's end) is two 4-row gathers (tile::gather4).  Rows past
-        // n repeat row n-1 (they are masked).
+        // boxes l / 16, l / 16 + 2, ...  The rows of a position tile are runs of consecutive
+        // rows of the buffer, one per chunk.  An aligned block of 2^s groups (s = 4 .. 0)
+        // that lies inside one run is one box of 8 << s rows, issued by the block's first
+        // lane and landing at the block's 1024-byte-aligned offset, so that the swizzled
+        // layout is the full box's; a group in no such block (it crosses a chunk boundary or
+        // the tile's end) is two 4-row gathers (tile::gather4).  Rows past n repeat row n-1
+        // (they are masked).
         const bool is_k = warp == 0;
         // this lane's group of 8 rows of a position tile (the indices are loaded one tile
         // ahead, so that the load latency overlaps the wait for a free stage)
@@ -220,18 +222,32 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
             for (int i = 0; i < 8; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(g8 + i, n - 1));
         };
         // 64-column boxes c0 .. c1-1 of those rows; a row r of the buffer is (r, head) of the
-        // 3-D map box8 and row r * heads + head of the row map
-        auto load_groups = [&](const CUtensorMap* box8, const CUtensorMap* rows, uint32_t dst, uint32_t bar,
-                               const int (&rr)[8], int heads, int head, int c0, int c1) {
+        // 3-D maps (full: 128-row boxes, runs[s]: 8 << s rows) and row r * heads + head of the
+        // row map.  Called by the whole warp.
+        auto load_groups = [&](const CUtensorMap* full, const CUtensorMap* runs, const CUtensorMap* rows,
+                               uint32_t dst, uint32_t bar, const int (&rr)[8], int heads, int head, int c0, int c1) {
+            const int g = lane & 15;
             bool run = true;
 #pragma unroll
             for (int i = 1; i < 8; ++i) run = run && rr[i] == rr[0] + i;
-            const uint32_t gdst = dst + (lane & 15) * 1024;
+            // bit g: group g is a run; bit g of link: group g+1 continues it (both halves of
+            // the warp hold the same groups, so the low 16 bits say it all)
+            const int next0 = __shfl_down_sync(0xffffffffu, rr[0], 1);
+            const uint32_t is_run = __ballot_sync(0xffffffffu, run) & 0xffffu;
+            const uint32_t link = __ballot_sync(0xffffffffu, run && next0 == rr[0] + 8) & (is_run >> 1) & 0x7fffu;
+            int size = -1;  // log2 of the groups in this lane's box; -1: gathers; -2: covered by another lane
+#pragma unroll
+            for (int s = 4; s >= 0 && size == -1; --s) {
+                const int n = 1 << s, b = g & ~(n - 1);
+                const uint32_t need_run = ((1u << n) - 1u) << b, need_link = ((1u << (n - 1)) - 1u) << b;
+                if ((is_run & need_run) == need_run && (link & need_link) == need_link) size = (g == b) ? s : -2;
+            }
+            const uint32_t gdst = dst + g * 1024;
             for (int c = c0 + (lane >> 4); c < c1; c += 2) {
                 const uint32_t d = gdst + c * L::kBox;
-                if (run) {
-                    tma_load_3d(box8, d, bar, (c - c0) * 64, head, rr[0]);
-                } else {
+                if (size >= 0) {
+                    tma_load_3d(size == 4 ? full : runs + size, d, bar, (c - c0) * 64, head, rr[0]);
+                } else if (size == -1) {
                     tma_gather4(rows, d, bar, (c - c0) * 64, rr[0] * heads + head, rr[1] * heads + head,
                                 rr[2] * heads + head, rr[3] * heads + head);
                     tma_gather4(rows, d + 512, bar, (c - c0) * 64, rr[4] * heads + head, rr[5] * heads + head,
@@ -307,7 +323,7 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
                     if (lane == 0)
                         for (int c = 0; c < DQK / 64; ++c) tma_load_3d(&tm.q, sQ + c * L::kBox, qf, c * 64, x.h, x.q0.z);
                 } else {
-                    load_groups(&tm.q8, &tm.qg, sQ, qf, rq, a.hq, x.h, 0, DQK / 64);
+                    load_groups(&tm.q, tm.qs, &tm.qg, sQ, qf, rq, a.hq, x.h, 0, DQK / 64);
                 }
             }
             for (int j = 0; j < nk; ++j) {
@@ -338,10 +354,10 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
                                     tma_load_3d(&tm.k, sK + st * L::kKBytes + c * L::kBox, kf, c * 64, x.g, box_row);
                             }
                     } else if (SHARED_ROPE) {  // per-head part, then the shared rope key (one row per token)
-                        load_groups(&tm.k8, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, 2);
-                        load_groups(&tm.kr8, &tm.krg, sK + st * L::kKBytes, kf, rr, 1, 0, 2, 3);
+                        load_groups(&tm.k, tm.ks, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, 2);
+                        load_groups(&tm.kr, tm.krs, &tm.krg, sK + st * L::kKBytes, kf, rr, 1, 0, 2, 3);
                     } else {
-                        load_groups(&tm.k8, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, DQK / 64);
+                        load_groups(&tm.k, tm.ks, &tm.kg, sK + st * L::kKBytes, kf, rr, a.hkv, x.g, 0, DQK / 64);
                     }
                 } else {
                     if (Jj >= NV)
@@ -355,7 +371,7 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
                             for (int c = 0; c < DV / 64; ++c)
                                 tma_load_3d(&tm.v, sV + st * L::kVBytes + c * L::kBox, vf, c * 64, x.g, box_row);
                     } else {
-                        load_groups(&tm.v8, &tm.vg, sV + st * L::kVBytes, vf, rr, a.hkv, x.g, 0, DV / 64);
+                        load_groups(&tm.v, tm.vs, &tm.vg, sV + st * L::kVBytes, vf, rr, a.hkv, x.g, 0, DV / 64);
                     }
                 }
             }

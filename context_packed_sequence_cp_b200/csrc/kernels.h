@@ -57,12 +57,13 @@ struct FwdArgs {
 };
 // Tensor maps of the bf16 forward, over Q [T, hq, dqk], K [T, hkv, dqk], V [T, hkv, dv]
 // (and K_rope [T, 1, 64] of the compact multi-head latent attention form, else K again):
-//   q, k, v, kr      3-D {dim, heads, rows} maps, boxes of 64 columns x 128 rows;
-//   q8, k8, v8, kr8  the same with boxes of 8 rows (runs inside position tiles);
-//   qg, kg, vg, krg  2-D {dim, rows * heads} row maps, boxes of one row (tile::gather4).
+//   q, k, v, kr          3-D {dim, heads, rows} maps, boxes of 64 columns x 128 rows;
+//   qs, ks, vs, krs [s]  the same with boxes of 8 << s rows (runs inside position tiles);
+//   qg, kg, vg, krg      2-D {dim, rows * heads} row maps, boxes of one row (tile::gather4).
+constexpr int kRunBoxes = 4;  // 8, 16, 32 and 64 rows
 struct FwdMaps {
     CUtensorMap q, k, v, kr;
-    CUtensorMap q8, k8, v8, kr8;
+    CUtensorMap qs[kRunBoxes], ks[kRunBoxes], vs[kRunBoxes], krs[kRunBoxes];
     CUtensorMap qg, kg, vg, krg;
 };
 int launch_fwd_sm100(int dqk, int dv, const FwdMaps& m, const FwdArgs& a, int n_items, cudaStream_t stream);
