@@ -142,6 +142,36 @@ def test_fwd_bf16_position_tiles_around_the_chunk_threshold(cp):
     assert np.abs(lse - want_l).max() <= LSE_MAX
 
 
+@pytest.mark.parametrize("cp", [2, 8])
+def test_fwd_bf16_position_tiles_run_boxes(cp):
+    """A position tile's rows are runs of consecutive rank-major rows, one per chunk, loaded
+    as the largest aligned boxes of 8 to 128 rows that lie inside one run, the rest gathered
+    4 rows at a time.  Chunk sizes 8, 16, 24, 32, 40, 64, 96, 120 put every run boundary on
+    an 8-row group boundary (boxes of every size); 9, 65, 127 put groups across chunk
+    boundaries (gathers mixed with boxes).  Every output is compared with the oracle, and the
+    fused-gather entry (K/V from the packed tensors) is bit-identical."""
+    import context_packed_sequence_cp_b200 as thd
+    from tests.gpu_util import unpermute_rows
+    chunks = [8, 16, 24, 32, 40, 64, 96, 120, 9, 65, 127]
+    cu = syn.cu_seqlens_of([2 * cp * c for c in chunks])
+    q, k, v = syn.make_tensors(int(cu[-1]), 8, 2, 128, 128, torch.bfloat16, seed=80 + cp, device="cuda")
+    plan = thd.Plan(cu, cp).upload()
+    assert (plan.export_fwd()["fqtiles"][:, 2] < 0).all()   # position tiles only
+    q_rm = thd.thd_kv_gather(plan, q)
+    k_rm, v_rm = thd.thd_kv_gather(plan, k, v)
+    o_rm, l_rm = thd.thd_cp_attn_fwd(plan, q_rm, k_rm, v_rm)
+    o_fg, l_fg = thd.thd_cp_attn_fwd_fused_gather(plan, q_rm, k, v)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    assert torch.equal(o_fg, o_rm) and torch.equal(l_fg, l_rm)
+    q_idx = plan.export()["q_idx"]
+    o = unpermute_rows(o_rm.float().cpu().numpy(), q_idx)
+    lse = unpermute_rows(l_rm.cpu().numpy().T, q_idx).T
+    want_o, want_l = A.attention_fwd(q.cpu(), k.cpu(), v.cpu(), cu, 1 / math.sqrt(128))
+    assert_bf16_close(o, want_o, "O")
+    assert np.abs(lse - want_l).max() <= LSE_MAX
+
+
 @pytest.mark.parametrize("cp,chunks,heads", [(4, [1, 17, 64, 127, 128, 129, 300, 3], (8, 2)),
                                               (16, [160, 32, 200], (8, 1)), (1, [900, 5], (4, 4))])
 def test_fwd_fused_gather_is_bit_identical(cp, chunks, heads):
