@@ -407,10 +407,16 @@ namespace {
 // of an item and overlaps with the neighbouring items.  With long items one CTA per item
 // measured as fast or faster, so the plan's mean key tiles per query tile decides.
 constexpr int64_t kPersistMaxMeanTiles = 64;
+// Item order.  Key/value group outermost keeps one group's K/V in L2 while its items run;
+// query tiles outermost (longest first over every group) balances the SMs better, since no
+// group's longest items start last, but its items in flight read one document's K/V for
+// every key/value head at once.  That order is taken when that much K/V (the longest
+// document's, all heads) fits in half of the 126 MB L2.
+constexpr int64_t kQtileOuterMaxDocKvBytes = 64ll << 20;
 
 // Arguments of the bf16 forward over the forward tables.
-thd::FwdArgs fwd_args(thd_plan* plan, void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, float scale,
-                      int32_t kv_global) {
+thd::FwdArgs fwd_args(thd_plan* plan, void* o_rm, float* lse_rm, int32_t hq, int32_t hkv, int32_t dk, int32_t dv,
+                      float scale, int32_t kv_global) {
     thd::FwdArgs a;
     a.qtiles = plan->d_fqtiles;
     a.entries = plan->d_fentries;
@@ -418,6 +424,8 @@ thd::FwdArgs fwd_args(thd_plan* plan, void* o_rm, float* lse_rm, int32_t hq, int
     a.rm_of_global = plan->d_rm_of_global;
     a.kv_global = kv_global;
     a.persistent = plan->n_fentries() < kPersistMaxMeanTiles * plan->n_fqtiles() ? 1 : 0;
+    const int64_t max_doc = plan->doc_len.empty() ? 0 : *std::max_element(plan->doc_len.begin(), plan->doc_len.end());
+    a.qtile_outer = max_doc * hkv * (dk + dv) * 2 <= kQtileOuterMaxDocKvBytes ? 1 : 0;
     a.o = static_cast<__nv_bfloat16*>(o_rm);
     a.lse = lse_rm;
     a.hq = hq;
@@ -446,7 +454,8 @@ int thd_cp_attn_fwd_mla(thd_cp_plan_t plan, const void* q_rm, const void* k_nope
     thd::FwdMaps maps;
     if (!make_fwd_maps(&maps, plan->T, q_rm, hq, d_nope + d_rope, k_nope_rm, hkv, d_nope, v_rm, dv, k_rope_rm, d_rope))
         return THD_ERR_CUDA;
-    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);  // the forward tables
+    // the forward tables; K is the per-head part plus the shared rope key
+    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, d_nope + d_rope, dv, scale, 0);
     if (items == 0) return THD_OK;
     return thd::launch_fwd_mla_sm100(maps, a, (int)items, static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA
@@ -471,7 +480,7 @@ int thd_cp_attn_fwd(thd_cp_plan_t plan, const void* q_rm, const void* k_rm, cons
         thd::FwdMaps maps;
         if (!make_fwd_maps(&maps, plan->T, q_rm, hq, dqk, k_rm, hkv, dqk, v_rm, dv, nullptr, 0)) return THD_ERR_CUDA;
         // the forward tables: rank-major tiles, position tiles for short-chunk documents
-        const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 0);
+        const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, dqk, dv, scale, 0);
         const int64_t fitems = plan->n_fqtiles() * (int64_t)hq;
         if (fitems == 0) return THD_OK;
         return thd::launch_fwd_sm100(dqk, dv, maps, a, (int)fitems, s) ? THD_ERR_CUDA : THD_OK;
@@ -511,7 +520,7 @@ int thd_cp_attn_fwd_fused_gather(thd_cp_plan_t plan, const void* q_rm, const voi
     if (items > INT32_MAX) return THD_ERR_INVALID_ARG;
     thd::FwdMaps maps;
     if (!make_fwd_maps(&maps, plan->T, q_rm, hq, dqk, k, hkv, dqk, v, dv, nullptr, 0)) return THD_ERR_CUDA;
-    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, scale, 1);
+    const thd::FwdArgs a = fwd_args(plan, o_rm, lse_rm, hq, hkv, dqk, dv, scale, 1);
     if (items == 0) return THD_OK;
     return thd::launch_fwd_sm100(dqk, dv, maps, a, (int)items, static_cast<cudaStream_t>(stream))
                ? THD_ERR_CUDA

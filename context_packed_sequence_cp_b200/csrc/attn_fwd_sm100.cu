@@ -85,7 +85,9 @@ static_assert(sizeof(Bars) <= 256, "barrier block");
 // A work item: one query tile and one query head.  Items are numbered key/value group
 // outermost, then query tiles longest-first, then the query heads of the group, so that
 // the items in flight together walk the K/V tiles of one group (a working set that stays
-// in L2) instead of all groups at once.  The grid has one CTA index per item.
+// in L2) instead of all groups at once; or, when a group has too few items to fill the
+// GPU (qtile_outer), query tiles longest-first outermost and every query head inner, so
+// that the longest items of every group start first.  The grid has one CTA per item.
 struct FwdItem {
     int h, g;
     int4 q0, q1, q2;  // the tile record: r, d, row0, m | qpos0, qbrk, qjump, qpos_max | nk, entry_off, ..
@@ -93,12 +95,20 @@ struct FwdItem {
 
 __device__ __forceinline__ FwdItem fwd_item(int it, const FwdArgs& a) {
     const int group = a.hq / a.hkv;
-    const int per_group = (int)(gridDim.x / (unsigned)a.hkv);  // query tiles x group
     FwdItem x;
-    x.g = it / per_group;
-    const int rem = it - x.g * per_group;
-    x.h = x.g * group + rem % group;
-    const int4* Q = reinterpret_cast<const int4*>(a.qtiles + (size_t)__ldg(a.lpt + rem / group) * 12);
+    int qr;  // rank of the query tile in the longest-first order
+    if (a.qtile_outer) {
+        qr = it / a.hq;
+        x.h = it - qr * a.hq;
+        x.g = x.h / group;
+    } else {
+        const int per_group = (int)(gridDim.x / (unsigned)a.hkv);  // query tiles x group
+        x.g = it / per_group;
+        const int rem = it - x.g * per_group;
+        x.h = x.g * group + rem % group;
+        qr = rem / group;
+    }
+    const int4* Q = reinterpret_cast<const int4*>(a.qtiles + (size_t)__ldg(a.lpt + qr) * 12);
     x.q0 = __ldg(Q);
     x.q1 = __ldg(Q + 1);
     x.q2 = __ldg(Q + 2);

@@ -48,6 +48,7 @@ struct FwdArgs {
     const int32_t* rm_of_global;  // rows of position tiles (row0 / k0 < 0)
     int32_t kv_global;            // K/V given in packed (global) order: rows are positions
     int32_t persistent;           // CTAs take over the items of CTAs that have not started
+    int32_t qtile_outer;          // item order: query tiles longest-first outermost (else kv group)
     __nv_bfloat16* o;
     float* lse;
     int32_t hq, hkv;
