@@ -7,11 +7,13 @@
 // and expanded MLA.  Section "Does this PR introduce any user-facing change?":
 // causal attention with EOD reset.
 //
-// A work item is one (query tile, query head); items are ordered by key/value group,
-// then longest-first, then query head, and the grid has one CTA per item.  CTAs are
-// persistent: each takes over the items of CTAs that have not started yet (cluster
-// launch control), keeping its TMEM and pipelines.  Warp roles (384 threads):
-//   warp 0      TMA producer of the Q tile and of K of every listed entry;
+// A work item is one (query tile, query head); the grid has one CTA per item, in one of
+// two orders (fwd_item).  Two instantiations: PERSIST, where a CTA takes over the items of
+// CTAs that have not started yet (cluster launch control) and keeps its TMEM and pipelines
+// (plans of short query tiles), and one CTA per item.  Warp roles (384 threads):
+//   warp 0      TMA producer of the Q tile and of K of every listed entry (position
+//               tiles: aligned boxes over runs of consecutive rows, 4-row gathers
+//               across chunk boundaries);
 //   warp 2      TMA producer of V (separate K and V rings, 128-byte swizzled
 //               boxes of 64 columns); a stage is refilled once the MMA that read
 //               it retired (K on the S signal, V on the PV signal).
@@ -30,7 +32,8 @@
 //               two halves' maxima meet in shared memory once per tile), writes its
 //               P_j columns as bf16 over S_j, and rescales its half of O in TMEM only
 //               when the running max grows by more than 2^8 (lazy correction);
-//               finally O / l and lse to global memory.
+//               finally O / l (whole 128-byte half rows after a lane transpose) and lse
+//               to global memory.
 // TMEM columns: [0,128) S0/P0, [128,256) S1/P1, [256,384) S2/P2, [384,384+DV) O.
 #include <cuda_bf16.h>
 
