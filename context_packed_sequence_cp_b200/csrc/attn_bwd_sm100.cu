@@ -468,11 +468,12 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_ld32(tY + lane_addr + hf * 64, v);
             tmem_wait_ld();
             stage(v);
+            // the first half goes to the TMA unit while the second is read out of TMEM
+            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
-            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             stage_free();
             stage(v);
             reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
