@@ -65,17 +65,6 @@ __device__ __forceinline__ StepMeta load_meta(const int32_t* kt_list, const int3
     return mt;
 }
 
-// Number of leading key columns of an entry a query at position qpos can see
-// (key t sits at kpos0 + t + (t >= kbrk ? kjump : 0); positions grow with t).
-__device__ __forceinline__ int visible_keys(int qpos, int nvalid, int kpos0, int kbrk, int kjump) {
-    if (qpos < kpos0) return 0;
-    const int a = min(kbrk, qpos - kpos0 + 1);
-    if (a < kbrk || kbrk >= nvalid) return min(a, nvalid);
-    const int b0 = kpos0 + kbrk + kjump;
-    if (qpos < b0) return kbrk;
-    return min(nvalid, kbrk + (qpos - b0 + 1));
-}
-
 // ---------------------------------------------------------------- prep
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
