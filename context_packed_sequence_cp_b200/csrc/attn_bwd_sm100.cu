@@ -137,13 +137,16 @@ struct FusedBars {
     int abort;
 };
 
+// Tensor maps of the fused kernel: q, k, v, dout with 64-column x 128-row boxes; the same
+// with 8 << s rows (runs inside position tiles, s = 0..3); 2-D row maps with one-row boxes
+// (tile::gather4); dq, dk, dv: fp32 32 x 32 boxes for the TMA reductions.
+struct BwdMaps {
+    CUtensorMap q, k, v, dout, dq, dk, dv, qg, kg, vg, dog;
+    CUtensorMap qs[kRunBoxes], ks[kRunBoxes], vs[kRunBoxes], dos[kRunBoxes];
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
-                 const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmQg,
-                 const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmVg,
-                 const __grid_constant__ CUtensorMap tmDOg, BwdArgs a) {
+bwd_fused_kernel(const __grid_constant__ BwdMaps tm, BwdArgs a) {
     using L = FusedLayout;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -218,26 +221,52 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (warp == 0) {
         // ---------------------------------------------------- producer warp
         const float log2e = 1.4426950408889634f;
-        // rank-major rows of this lane's 4 rows (4 lane .. 4 lane + 3) of a position tile,
-        // rows past n repeating row n-1
-        auto position_rows = [&](int pos0, int n, int (&rr)[4]) {
+        // A position tile's rows (positions pos0 .. pos0+n-1, rows past n repeating row n-1)
+        // are runs of consecutive rank-major rows, one per chunk.  Lane l takes the group of
+        // 8 tile rows l % 16 and the 64-column box l / 16; an aligned block of 2^s groups
+        // inside one run is one box of 8 << s rows issued by its first lane (landing at the
+        // block's 1024-byte-aligned offset, the full box's swizzled layout), any other group
+        // two 4-row gathers.
+        auto group_index = [&](int pos0, int n, int (&rr)[8]) {
+            const int g8 = (lane & 15) * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(lane * 4 + i, n - 1));
+            for (int i = 0; i < 8; ++i) rr[i] = __ldg(a.rm_of_global + pos0 + min(g8 + i, n - 1));
         };
-        auto gather = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, const int (&rr)[4], int heads, int head) {
+        auto load_groups = [&](const CUtensorMap* full, const CUtensorMap* runs, const CUtensorMap* rows,
+                               uint32_t dst, uint32_t bar, const int (&rr)[8], int heads, int head) {
+            const int gq = lane & 15;
+            bool run = true;
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                tma_gather4(map, dst + c * kBox + lane * 512, bar, c * 64, rr[0] * heads + head, rr[1] * heads + head,
-                            rr[2] * heads + head, rr[3] * heads + head);
+            for (int i = 1; i < 8; ++i) run = run && rr[i] == rr[0] + i;
+            const int next0 = __shfl_down_sync(0xffffffffu, rr[0], 1);
+            const uint32_t is_run = __ballot_sync(0xffffffffu, run) & 0xffffu;
+            const uint32_t link = __ballot_sync(0xffffffffu, run && next0 == rr[0] + 8) & (is_run >> 1) & 0x7fffu;
+            int size = -1;  // log2 of the groups in this lane's box; -1: gathers; -2: covered by another lane
+#pragma unroll
+            for (int sz = 4; sz >= 0 && size == -1; --sz) {
+                const int n = 1 << sz, b = gq & ~(n - 1);
+                const uint32_t need_run = ((1u << n) - 1u) << b, need_link = ((1u << (n - 1)) - 1u) << b;
+                if ((is_run & need_run) == need_run && (link & need_link) == need_link) size = (gq == b) ? sz : -2;
+            }
+            const int c = lane >> 4;
+            const uint32_t d = dst + c * kBox + gq * 1024;
+            if (size >= 0) {
+                tma_load_3d(size == 4 ? full : runs + size, d, bar, c * 64, head, rr[0]);
+            } else if (size == -1) {
+                tma_gather4(rows, d, bar, c * 64, rr[0] * heads + head, rr[1] * heads + head, rr[2] * heads + head,
+                            rr[3] * heads + head);
+                tma_gather4(rows, d + 512, bar, c * 64, rr[4] * heads + head, rr[5] * heads + head,
+                            rr[6] * heads + head, rr[7] * heads + head);
+            }
         };
         if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            tma_prefetch_desc(&tmDO);
-            tma_prefetch_desc(&tmDQ);
-            tma_prefetch_desc(&tmDK);
-            tma_prefetch_desc(&tmDV);
+            tma_prefetch_desc(&tm.q);
+            tma_prefetch_desc(&tm.k);
+            tma_prefetch_desc(&tm.v);
+            tma_prefetch_desc(&tm.dout);
+            tma_prefetch_desc(&tm.dq);
+            tma_prefetch_desc(&tm.dk);
+            tma_prefetch_desc(&tm.dv);
         }
         const uint32_t kvf = smem_u32(&bars->kv_full);
         if (lane == 0) mbar_arrive_expect_tx(kvf, 2 * kTile);
@@ -245,18 +274,18 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (k0 >= 0) {
             if (lane == 0)
                 for (int c = 0; c < 2; ++c) {
-                    tma_load_3d(&tmK, sK + c * kBox, kvf, c * 64, g, k0);
-                    tma_load_3d(&tmV, sV + c * kBox, kvf, c * 64, g, k0);
+                    tma_load_3d(&tm.k, sK + c * kBox, kvf, c * 64, g, k0);
+                    tma_load_3d(&tm.v, sV + c * kBox, kvf, c * 64, g, k0);
                 }
         } else {
-            int rk[4];
-            position_rows(kpos0, kn, rk);
-            gather(&tmKg, sK, kvf, rk, a.hkv, g);
-            gather(&tmVg, sV, kvf, rk, a.hkv, g);
+            int rk[8];
+            group_index(kpos0, kn, rk);
+            load_groups(&tm.k, tm.ks, &tm.kg, sK, kvf, rk, a.hkv, g);
+            load_groups(&tm.v, tm.vs, &tm.vg, sV, kvf, rk, a.hkv, g);
         }
         StepMeta cur = load_meta(kt_list, qtiles, entries, l0), nxt = cur;
         if (llen > 1) nxt = load_meta(kt_list, qtiles, entries, l0 + 1);
-        int rq[4] = {0, 0, 0, 0};   // gathered rows of the current query tile (position tiles)
+        int rq[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // this lane's rows of the current query tile (position tiles)
         int rs[4] = {0, 0, 0, 0};   // rank-major rows of lse / Delta entries lane + 32 u (-1: none)
         for (int it = 0; it < n_it; ++it) {
             const int pos = it / group, hh = it - pos * group;   // query tiles outer, heads inner
@@ -273,7 +302,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                     rs[u] = row0 >= 0 ? (row0 + t < a.T ? row0 + t : -1)
                                       : (t < cur.m ? __ldg(a.rm_of_global + cur.qpos0 + t) : -1);
                 }
-                if (row0 < 0) position_rows(cur.qpos0, cur.m, rq);
+                if (row0 < 0) group_index(cur.qpos0, cur.m, rq);
             }
             float lv[4], dv[4];
 #pragma unroll
@@ -292,9 +321,9 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __syncwarp();
             if (row0 >= 0) {
                 if (lane == 0)
-                    for (int c = 0; c < 2; ++c) tma_load_3d(&tmDO, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
+                    for (int c = 0; c < 2; ++c) tma_load_3d(&tm.dout, sDO + st * kTile + c * kBox, f, c * 64, h, row0);
             } else {
-                gather(&tmDOg, sDO + st * kTile, f, rq, a.hq, h);
+                load_groups(&tm.dout, tm.dos, &tm.dog, sDO + st * kTile, f, rq, a.hq, h);
             }
             float* stat = s_stat + st * 256;
 #pragma unroll
@@ -310,9 +339,9 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             __syncwarp();
             if (row0 >= 0) {
                 if (lane == 0)
-                    for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, sQ + st * kTile + c * kBox, qf, c * 64, h, row0);
+                    for (int c = 0; c < 2; ++c) tma_load_3d(&tm.q, sQ + st * kTile + c * kBox, qf, c * 64, h, row0);
             } else {
-                gather(&tmQg, sQ + st * kTile, qf, rq, a.hq, h);
+                load_groups(&tm.q, tm.qs, &tm.qg, sQ + st * kTile, qf, rq, a.hq, h);
             }
         }
     } else if (warp == 1) {
@@ -458,14 +487,14 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_wait_ld();
             stage(v);
             // the first half goes to the TMA unit while the second is read out of TMEM
-            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
+            reduce(&tm.dq, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
             stage_free();
             stage(v);
-            reduce(&tmDQ, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
+            reduce(&tm.dq, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
         };
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
@@ -581,7 +610,7 @@ bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tmem_wait_ld();
                 stage_free();
                 stage(v);
-                reduce(which == 0 ? &tmDK : &tmDV, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kpos0, kn, hf * 64 + ch * 32);
+                reduce(which == 0 ? &tm.dk : &tm.dv, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kpos0, kn, hf * 64 + ch * 32);
             }
         }
         stage_free();   // every box read before the CTA's shared memory is released
@@ -599,18 +628,26 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
     if (dqk != kD || dv != kD) return -2;
     static std::atomic<uint64_t> configured{0};
     if (!ensure_dynamic_smem(bwd_fused_kernel, FusedLayout::kBytes, configured)) return -1;
-    CUtensorMap mdq, mdk, mdv, mqg, mkg, mvg, mdog;
-    if (!make_map_f32_box32(&mdq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&mdk, a.dk, a.T, a.hkv, kD) ||
-        !make_map_f32_box32(&mdv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&mqg, a.q, a.T * a.hq, kD) ||
-        !make_map_bf16_rows(&mkg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&mvg, a.v, a.T * a.hkv, kD) ||
-        !make_map_bf16_rows(&mdog, a.dout, a.T * a.hq, kD))
+    BwdMaps m;
+    m.q = q;
+    m.k = k;
+    m.v = v;
+    m.dout = dout;
+    if (!make_map_f32_box32(&m.dq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&m.dk, a.dk, a.T, a.hkv, kD) ||
+        !make_map_f32_box32(&m.dv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&m.qg, a.q, a.T * a.hq, kD) ||
+        !make_map_bf16_rows(&m.kg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&m.vg, a.v, a.T * a.hkv, kD) ||
+        !make_map_bf16_rows(&m.dog, a.dout, a.T * a.hq, kD))
         return -1;
+    for (int s = 0; s < kRunBoxes; ++s)
+        if (!make_map_bf16(&m.qs[s], a.q, a.T, a.hq, kD, 8 << s) || !make_map_bf16(&m.ks[s], a.k, a.T, a.hkv, kD, 8 << s) ||
+            !make_map_bf16(&m.vs[s], a.v, a.T, a.hkv, kD, 8 << s) ||
+            !make_map_bf16(&m.dos[s], a.dout, a.T, a.hq, kD, 8 << s))
+            return -1;
     bwd_prep_kernel<<<num_sms * 8, 256, 0, stream>>>(a.o, a.dout, a.delta, a.dq_acc, a.dk, a.dv, a.T * a.hkv,
                                                      a.T * a.hq, a.hq, a.T);
     if (cudaGetLastError() != cudaSuccess) return -1;
     const unsigned items = (unsigned)((int64_t)n_items_per_group * a.hkv);
-    bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(q, k, v, dout, mdq, mdk, mdv, mqg, mkg, mvg,
-                                                                       mdog, a);
+    bwd_fused_kernel<<<items, kThreads, FusedLayout::kBytes, stream>>>(m, a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
