@@ -194,12 +194,12 @@ bool make_fwd_maps(thd::FwdMaps* m, int64_t T, const void* q, int hq, int dqk, c
            make_map_bf16_rows(&m->vg, v, T * hkv, dv) && make_map_bf16_rows(&m->krg, kr, T * hr, dr);
 }
 
-bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim) {
+bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)dim, (cuuint64_t)heads, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)dim * 4, (cuuint64_t)heads * dim * 4};
-    const cuuint32_t box[3] = {32, 1, 32};
+    const cuuint32_t box[3] = {32, 1, (cuuint32_t)box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

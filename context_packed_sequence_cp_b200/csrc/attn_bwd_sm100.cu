@@ -139,9 +139,10 @@ struct FusedBars {
 
 // Tensor maps of the fused kernel: q, k, v, dout with 64-column x 128-row boxes; the same
 // with 8 << s rows (runs inside position tiles, s = 0..3); 2-D row maps with one-row boxes
-// (tile::gather4); dq, dk, dv: fp32 32 x 32 boxes for the TMA reductions.
+// (tile::gather4); dq, dk, dv: fp32 32 x 32 boxes for the TMA reductions, dq8, dk8, dv8 the
+// same 8 rows high.
 struct BwdMaps {
-    CUtensorMap q, k, v, dout, dq, dk, dv, qg, kg, vg, dog;
+    CUtensorMap q, k, v, dout, dq, dk, dv, qg, kg, vg, dog, dq8, dk8, dv8;
     CUtensorMap qs[kRunBoxes], ks[kRunBoxes], vs[kRunBoxes], dos[kRunBoxes];
 };
 
@@ -450,10 +451,14 @@ bwd_fused_kernel(const __grid_constant__ BwdMaps tm, BwdArgs a) {
             __syncwarp();
         };
         // adds the staged box at (row0 + 32 wq, head, col) of a [rows, heads, 128] fp32
-        // tensor with `valid` rows from row0 on; a position tile (row0 < 0) adds its rows
-        // (positions pos0 ..) one by one at their rank-major rows
-        auto reduce = [&](const CUtensorMap* map, float* gbase, int heads, int head, int row0, int pos0, int valid,
-                          int col) {
+        // tensor with `valid` rows from row0 on.  A position tile (row0 < 0; rows at positions
+        // pos0 .., found through rm_of_global) or a short tile adds every aligned group of 8
+        // rows that are 8 consecutive rows of the tensor as an 8-row sub-box (map8: its staged
+        // rows start at a 1024-byte boundary, the box's swizzled layout), the other rows one by
+        // one with vector reductions.  Only lane 0 issues bulk operations, so that its wait
+        // covers every box of the warp.
+        auto reduce = [&](const CUtensorMap* map, const CUtensorMap* map8, float* gbase, int heads, int head,
+                          int row0, int pos0, int valid, int col) {
             if (row0 >= 0 && wq * 32 + 32 <= valid) {
                 fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
                 __syncwarp();
@@ -462,15 +467,32 @@ bwd_fused_kernel(const __grid_constant__ BwdMaps tm, BwdArgs a) {
                     bulk_commit_group();
                 }
             } else {
+                const int q_l = wq * 32 + lane;
+                const int row_l = q_l < valid ? (row0 >= 0 ? row0 + q_l : __ldg(a.rm_of_global + pos0 + q_l)) : -1;
+                const int lead = __shfl_sync(0xffffffffu, row_l, lane & ~7);
+                const uint32_t ok = __ballot_sync(0xffffffffu, row_l >= 0 && row_l == lead + (lane & 7));
+                uint32_t runs = 0;  // bit k: rows 8k .. 8k+7 go as one sub-box
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (((ok >> (8 * k)) & 0xffu) == 0xffu) runs |= 1u << k;
+                if (runs) fence_proxy_async_smem();   // the staged rows, visible to the TMA unit
                 __syncwarp();
+                int r8[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) r8[k] = __shfl_sync(0xffffffffu, row_l, 8 * k);
+                if (lane == 0 && runs) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if ((runs >> k) & 1u) tma_reduce_add_3d(map8, warp_stage + k * 1024, col, head, r8[k]);
+                    bulk_commit_group();
+                }
                 const int sub = lane >> 3, chunk = lane & 7;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int rr = 4 * j + sub;
-                    const int q = wq * 32 + rr;
-                    if (q < valid) {
+                    const int row = __shfl_sync(0xffffffffu, row_l, rr);
+                    if (row >= 0 && !((runs >> (rr >> 3)) & 1u)) {
                         const float4 x = ld_shared_f4(warp_stage + rr * 128 + ((chunk ^ (rr & 7)) << 4));
-                        const int row = row0 >= 0 ? row0 + q : __ldg(a.rm_of_global + pos0 + q);
                         red_add_v4(gbase + ((int64_t)row * heads + head) * kD + col + 4 * chunk, x.x, x.y, x.z, x.w);
                     }
                 }
@@ -487,14 +509,14 @@ bwd_fused_kernel(const __grid_constant__ BwdMaps tm, BwdArgs a) {
             tmem_wait_ld();
             stage(v);
             // the first half goes to the TMA unit while the second is read out of TMEM
-            reduce(&tm.dq, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
+            reduce(&tm.dq, &tm.dq8, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64);
             tmem_ld32(tY + lane_addr + hf * 64 + 32, v);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->dq_free));   // Y read out: b(it+1) may overwrite it
             stage_free();
             stage(v);
-            reduce(&tm.dq, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
+            reduce(&tm.dq, &tm.dq8, a.dq_acc, a.hq, h, mt.row0, mt.qpos0, mt.m, hf * 64 + 32);
         };
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
@@ -610,7 +632,8 @@ bwd_fused_kernel(const __grid_constant__ BwdMaps tm, BwdArgs a) {
                 tmem_wait_ld();
                 stage_free();
                 stage(v);
-                reduce(which == 0 ? &tm.dk : &tm.dv, which == 0 ? a.dk : a.dv, a.hkv, g, k0, kpos0, kn, hf * 64 + ch * 32);
+                reduce(which == 0 ? &tm.dk : &tm.dv, which == 0 ? &tm.dk8 : &tm.dv8, which == 0 ? a.dk : a.dv, a.hkv, g,
+                       k0, kpos0, kn, hf * 64 + ch * 32);
             }
         }
         stage_free();   // every box read before the CTA's shared memory is released
@@ -634,7 +657,8 @@ int launch_bwd_sm100(int dqk, int dv, const CUtensorMap& q, const CUtensorMap& k
     m.v = v;
     m.dout = dout;
     if (!make_map_f32_box32(&m.dq, a.dq_acc, a.T, a.hq, kD) || !make_map_f32_box32(&m.dk, a.dk, a.T, a.hkv, kD) ||
-        !make_map_f32_box32(&m.dv, a.dv, a.T, a.hkv, kD) || !make_map_bf16_rows(&m.qg, a.q, a.T * a.hq, kD) ||
+        !make_map_f32_box32(&m.dv, a.dv, a.T, a.hkv, kD) || !make_map_f32_box32(&m.dq8, a.dq_acc, a.T, a.hq, kD, 8) ||
+        !make_map_f32_box32(&m.dk8, a.dk, a.T, a.hkv, kD, 8) || !make_map_f32_box32(&m.dv8, a.dv, a.T, a.hkv, kD, 8) || !make_map_bf16_rows(&m.qg, a.q, a.T * a.hq, kD) ||
         !make_map_bf16_rows(&m.kg, a.k, a.T * a.hkv, kD) || !make_map_bf16_rows(&m.vg, a.v, a.T * a.hkv, kD) ||
         !make_map_bf16_rows(&m.dog, a.dout, a.T * a.hq, kD))
         return -1;

@@ -32,7 +32,7 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int heads, 
 bool make_map_bf16_rows(CUtensorMap* map, const void* base, int64_t rows, int dim);
 // [rows, heads, dim] fp32 tensor viewed as a 3-D TMA map with 32-column x 1-head x 32-row
 // boxes (128-byte rows) and 128-byte swizzle: the target of tiled reductions.
-bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim);
+bool make_map_f32_box32(CUtensorMap* map, const void* base, int64_t rows, int heads, int dim, int box_rows = 32);
 
 // ---- row gather (all-gather layout, and its inverse) -----------------------
 // dst_t[j] = src_t[idx[j]] for whole rows of row_bytes_t bytes, t = 0, 1 (the second
