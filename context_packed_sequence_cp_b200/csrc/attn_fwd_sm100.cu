@@ -189,9 +189,10 @@ fwd_kernel(const __grid_constant__ FwdMaps tm, FwdArgs a) {
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    // Persistent CTAs.  After its own item (blockIdx.x) a CTA takes over the item of a CTA
-    // that has not started yet, by cancelling that CTA's launch (cluster launch control),
-    // until none is left.  Items are still taken in launch order, so the order above holds,
+    // Persistent CTAs (PERSIST; otherwise a CTA computes its own item only).  After its own
+    // item (blockIdx.x) a CTA takes over the item of a CTA that has not started yet, by
+    // cancelling that CTA's launch (cluster launch control), until none is left.  Items are
+    // still taken in launch order, so the item order of fwd_item holds,
     // and an SM keeps its CTA, TMEM and pipelines across items: the next item's loads and
     // first MMAs overlap the current item's last tiles and its epilogue.  Every barrier
     // phase below counts the tiles J of all the CTA's items so far.
